@@ -1,0 +1,160 @@
+"""float64 CPU oracle for the Hyena order-N forward (ctypes wrapper of oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by ``__graft_entry__.smoke()``
+and by the CPU-baseline leg of ``bench.py``. The CUDA library never imports
+or links it, and it never imports the CUDA library.
+
+What each function computes, and the passage it follows, is stated in
+oracle.c. Parity pins live in tests/test_oracle_pins.py. The implicit-filter
+FFN itself has no printed worked example on the pages; it is pinned only
+through closed-form special cases of its weights (see the pins).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "liboracle.so")
+
+DIRECT_MAX_L = 8192
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc (-O2, no fast-math: the summation order is
+    the one written in the source)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        l = ctypes.CDLL(build())
+        d, i64, i32 = ctypes.c_double, ctypes.c_int64, ctypes.c_int
+        P = ctypes.c_void_p
+        l.oracle_fft.argtypes = [P, P, i64, i32]
+        l.oracle_causal_conv_direct.argtypes = [P, P, i64, P]
+        l.oracle_causal_conv_fft.argtypes = [P, P, i64, P]
+        l.oracle_causal_conv.argtypes = [P, P, i64, P]
+        l.oracle_filter_spectrum.argtypes = [P, i64, P, P]
+        l.oracle_embedding.argtypes = [i32, i32, i32, P]
+        l.oracle_alpha.argtypes = [i32, i32, d, d]
+        l.oracle_alpha.restype = d
+        l.oracle_filter.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, d, d,
+                                    i32, P, P, P, i32]
+        l.oracle_hyena_forward.argtypes = [P, P, P, P, i64, i32, i64, i32, P, i32]
+        l.oracle_hyena_forward.restype = i32
+        _lib = l
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def default_threads() -> int:
+    return os.cpu_count() or 1
+
+
+def fft(x, sign: int = -1) -> np.ndarray:
+    """Unnormalised DFT, X[k] = sum x[n] exp(sign 2 pi i n k / n) (power-of-two n)."""
+    x = np.asarray(x, dtype=np.complex128)
+    re, im = _f64(x.real).copy(), _f64(x.imag).copy()
+    lib().oracle_fft(_p(re), _p(im), len(re), int(sign))
+    return re + 1j * im
+
+
+def causal_conv(h, z, method: str = "auto") -> np.ndarray:
+    """(h conv z)[t] = sum_{s<=t} h[t-s] z[s], t < L."""
+    h, z = _f64(h), _f64(z)
+    assert h.shape == z.shape and h.ndim == 1
+    out = np.empty_like(z)
+    fn = {"auto": lib().oracle_causal_conv, "direct": lib().oracle_causal_conv_direct,
+          "fft": lib().oracle_causal_conv_fft}[method]
+    fn(_p(h), _p(z), len(z), _p(out))
+    return out
+
+
+def filter_spectrum(h) -> np.ndarray:
+    """H[k] = sum_{t<L} h[t] exp(-2 pi i k t / 2L), k = 0..L (complex128, L+1 values)."""
+    h = _f64(h)
+    L = len(h)
+    re, im = np.empty(L + 1), np.empty(L + 1)
+    lib().oracle_filter_spectrum(_p(h), L, _p(re), _p(im))
+    return re + 1j * im
+
+
+def embedding(t: int, L: int, n_bands: int = 8) -> np.ndarray:
+    e = np.empty(1 + 2 * n_bands)
+    lib().oracle_embedding(int(t), int(L), int(n_bands), _p(e))
+    return e
+
+
+def alpha(c: int, D: int, lo: float, hi: float) -> float:
+    return lib().oracle_alpha(int(c), int(D), float(lo), float(hi))
+
+
+def implicit_filter(weights: dict, N: int, D: int, L: int, alpha_lo: float, alpha_hi: float,
+                    rows: list[tuple[int, int]] | None = None, n_bands: int = 8,
+                    threads: int | None = None) -> np.ndarray:
+    """h rows [len(rows)][L] for (n, c) pairs (n 0-based); all N*D rows in
+    [n][c] order when rows is None."""
+    W1, b1, W2, b2, W3, b3 = (_f32(weights[k]) for k in ("W1", "b1", "W2", "b2", "W3", "b3"))
+    width = W1.shape[0]
+    assert W1.shape == (width, 1 + 2 * n_bands) and W2.shape == (width, width)
+    assert W3.shape == (N * D, width) and b3.shape == (N * D,)
+    if rows is None:
+        rows = [(n, c) for n in range(N) for c in range(D)]
+    rn = np.ascontiguousarray([r[0] for r in rows], dtype=np.int32)
+    rc = np.ascontiguousarray([r[1] for r in rows], dtype=np.int32)
+    h = np.empty((len(rows), L))
+    lib().oracle_filter(_p(W1), _p(b1), _p(W2), _p(b2), _p(W3), _p(b3), n_bands, width,
+                        N, D, L, float(alpha_lo), float(alpha_hi), len(rows), _p(rn), _p(rc),
+                        _p(h), threads or default_threads())
+    return h
+
+
+def hyena_forward(v, xs, hs, filter_row=None, threads: int | None = None) -> np.ndarray:
+    """Order-N forward on independent channels.
+
+    v: [C][L]; xs: N arrays [C][L]; hs: N arrays [F][L] (filter rows);
+    filter_row: per channel the row of each h_n it uses (default: row r).
+    Returns y [C][L] (float64).
+    """
+    v = _f64(np.atleast_2d(v))
+    C, L = v.shape
+    N = len(xs)
+    x = _f64(np.stack([np.atleast_2d(a) for a in xs]))
+    h = _f64(np.stack([np.atleast_2d(a) for a in hs]))
+    assert x.shape == (N, C, L) and h.shape[0] == N and h.shape[2] == L
+    F = h.shape[1]
+    fr = np.ascontiguousarray(np.arange(C) if filter_row is None else filter_row, dtype=np.int32)
+    assert fr.shape == (C,) and (fr >= 0).all() and (fr < F).all()
+    y = np.empty((C, L))
+    rc = lib().oracle_hyena_forward(_p(v), _p(x), _p(h), _p(fr), C, F, L, N, _p(y),
+                                    threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_hyena_forward rejected its arguments")
+    return y

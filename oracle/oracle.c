@@ -1,0 +1,317 @@
+/*
+ * oracle.c -- float64 CPU oracle for the Hyena order-N forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and the
+ * CPU-baseline leg of bench.py may load this library. It shares no code,
+ * header, table or constant with the CUDA library: it is the plain
+ * definition of what that library computes, written so that it can be
+ * checked against the pages by eye.
+ *
+ * Sources (page title, section):
+ *  - Order-N recurrence z_1 = v, z_{n+1} = x_n * (h_n conv z_n), y = z_{N+1}:
+ *    "Hyena Hierarchy - Towards Larger Convolutional Language Models" digest,
+ *    section "방법 (Method) / 프레임워크 개요" (the framework graph); and the
+ *    explainer "Hyena Hierarchy: Towards Larger Convolutional Language
+ *    Models", section "Hyena 演算子の形".
+ *  - Causal convolution (h conv z)_t = sum_{s=0..t} h_{t-s} z_s: "02. 3つの
+ *    Hyena 演算子", section "4. FIR フィルタと効率的な生成" (the FIR sum).
+ *  - FFT evaluation on a 2L zero-padded grid: glossary "Hyena（ハイエナ）",
+ *    section "計算効率"; HyenaND summary, "境界の処理" (zero padding to twice
+ *    the grid avoids wrap-around leakage).
+ *  - Implicit filter h(t) = Window(t) * FFN(t/L, sin, cos): glossary
+ *    "Hyena（ハイエナ）", section "暗黙的畳み込みフィルタ". The exact recipe
+ *    (17-dim embedding, Linear-sin-Linear-sin-Linear, exp(-alpha_c t / L)
+ *    window with alpha_c linearly spaced) is the workload specification.
+ *
+ * Evaluation rules: direct O(L^2) causal sum for L <= 8192; above that a
+ * naive recursive radix-2 FFT on the 2L zero-padded grid, keeping the first
+ * L outputs. All arithmetic in double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_DIRECT_MAX_L 8192
+
+static const double ORACLE_PI = 3.14159265358979323846264338327950288;
+
+/* ------------------------------------------------------------------------ */
+/* Implicit filter                                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Positional embedding of tap t for a filter of length L:
+ *   e = [ t/L, sin(2 pi k t / L) for k = 1..K, cos(2 pi k t / L) for k = 1..K ]
+ * (1 + 2K values; block order: the linear term, then the K sines, then the
+ * K cosines).
+ */
+void oracle_embedding(int t, int L, int n_bands, double *e)
+{
+    e[0] = (double)t / (double)L;
+    for (int k = 1; k <= n_bands; ++k) {
+        double a = 2.0 * ORACLE_PI * (double)k * (double)t / (double)L;
+        e[k] = sin(a);
+        e[n_bands + k] = cos(a);
+    }
+}
+
+/* alpha_c linearly spaced over [lo, hi] with both ends included. */
+double oracle_alpha(int c, int D, double lo, double hi)
+{
+    if (D <= 1) return lo;
+    return lo + (hi - lo) * (double)c / (double)(D - 1);
+}
+
+typedef struct {
+    const float *W1, *b1, *W2, *b2, *W3, *b3;
+    int n_bands, width, N, D, L;
+    double alpha_lo, alpha_hi;
+    int n_rows;           /* number of (n, c) filter rows requested */
+    const int *rows_n;    /* filter index n in [0, N) */
+    const int *rows_c;    /* channel index c in [0, D) */
+    double *h;            /* [n_rows][L] */
+    int t_begin, t_end;
+} filter_job;
+
+static void *filter_worker(void *arg)
+{
+    filter_job *j = (filter_job *)arg;
+    const int E = 1 + 2 * j->n_bands, H = j->width;
+    double *e = (double *)malloc(sizeof(double) * E);
+    double *s1 = (double *)malloc(sizeof(double) * H);
+    double *s2 = (double *)malloc(sizeof(double) * H);
+    for (int t = j->t_begin; t < j->t_end; ++t) {
+        oracle_embedding(t, j->L, j->n_bands, e);
+        /* layer 1: s1 = sin(W1 e + b1), W1 is [H][E] row-major */
+        for (int o = 0; o < H; ++o) {
+            double acc = (double)j->b1[o];
+            for (int i = 0; i < E; ++i) acc += (double)j->W1[o * E + i] * e[i];
+            s1[o] = sin(acc);
+        }
+        /* layer 2: s2 = sin(W2 s1 + b2), W2 is [H][H] */
+        for (int o = 0; o < H; ++o) {
+            double acc = (double)j->b2[o];
+            for (int i = 0; i < H; ++i) acc += (double)j->W2[o * H + i] * s1[i];
+            s2[o] = sin(acc);
+        }
+        /* layer 3 and window: output column (n * D + c) is filter n, channel c */
+        for (int r = 0; r < j->n_rows; ++r) {
+            int n = j->rows_n[r], c = j->rows_c[r];
+            int o = n * j->D + c;
+            double acc = (double)j->b3[o];
+            for (int i = 0; i < H; ++i) acc += (double)j->W3[o * H + i] * s2[i];
+            double alpha = oracle_alpha(c, j->D, j->alpha_lo, j->alpha_hi);
+            double window = exp(-alpha * (double)t / (double)j->L);
+            j->h[(size_t)r * j->L + t] = acc * window;
+        }
+    }
+    free(e); free(s1); free(s2);
+    return NULL;
+}
+
+/*
+ * h[r][t] for the requested (n, c) rows, t in [0, L).
+ * Weights are the float32 values the GPU receives, evaluated in double.
+ */
+void oracle_filter(const float *W1, const float *b1, const float *W2, const float *b2,
+                   const float *W3, const float *b3, int n_bands, int width,
+                   int N, int D, int L, double alpha_lo, double alpha_hi,
+                   int n_rows, const int *rows_n, const int *rows_c,
+                   double *h, int n_threads)
+{
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > L) n_threads = L;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n_threads);
+    filter_job *jobs = (filter_job *)malloc(sizeof(filter_job) * n_threads);
+    for (int i = 0; i < n_threads; ++i) {
+        filter_job j = {W1, b1, W2, b2, W3, b3, n_bands, width, N, D, L, alpha_lo, alpha_hi,
+                        n_rows, rows_n, rows_c, h,
+                        (int)((int64_t)L * i / n_threads), (int)((int64_t)L * (i + 1) / n_threads)};
+        jobs[i] = j;
+        pthread_create(&th[i], NULL, filter_worker, &jobs[i]);
+    }
+    for (int i = 0; i < n_threads; ++i) pthread_join(th[i], NULL);
+    free(th); free(jobs);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Naive recursive radix-2 FFT                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * In place, unnormalised: X[k] = sum_n x[n] exp(sign * 2 pi i n k / n_pts),
+ * sign = -1 forward, +1 inverse. n_pts must be a power of two. Textbook
+ * decimation in time: split even/odd samples, transform each half, combine
+ * X[k] = E[k] + w^k O[k], X[k + n/2] = E[k] - w^k O[k].
+ */
+void oracle_fft(double *re, double *im, int64_t n, int sign)
+{
+    if (n <= 1) return;
+    int64_t h = n / 2;
+    double *er = (double *)malloc(sizeof(double) * h), *ei = (double *)malloc(sizeof(double) * h);
+    double *or_ = (double *)malloc(sizeof(double) * h), *oi = (double *)malloc(sizeof(double) * h);
+    for (int64_t i = 0; i < h; ++i) {
+        er[i] = re[2 * i];     ei[i] = im[2 * i];
+        or_[i] = re[2 * i + 1]; oi[i] = im[2 * i + 1];
+    }
+    oracle_fft(er, ei, h, sign);
+    oracle_fft(or_, oi, h, sign);
+    for (int64_t k = 0; k < h; ++k) {
+        double ang = (double)sign * 2.0 * ORACLE_PI * (double)k / (double)n;
+        double wr = cos(ang), wi = sin(ang);
+        double tr = wr * or_[k] - wi * oi[k];
+        double ti = wr * oi[k] + wi * or_[k];
+        re[k] = er[k] + tr;      im[k] = ei[k] + ti;
+        re[k + h] = er[k] - tr;  im[k + h] = ei[k] - ti;
+    }
+    free(er); free(ei); free(or_); free(oi);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Causal long convolution                                                  */
+/* ------------------------------------------------------------------------ */
+
+/* out[t] = sum_{s=0..t} h[t-s] z[s], t in [0, L): the plain definition. */
+void oracle_causal_conv_direct(const double *h, const double *z, int64_t L, double *out)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        double acc = 0.0;
+        for (int64_t s = 0; s <= t; ++s) acc += h[t - s] * z[s];
+        out[t] = acc;
+    }
+}
+
+/* Same result via FFT: zero-pad both to 2L, transform, multiply pointwise,
+ * inverse transform, divide by 2L, keep the first L samples. */
+void oracle_causal_conv_fft(const double *h, const double *z, int64_t L, double *out)
+{
+    int64_t n = 2 * L;
+    double *hr = (double *)calloc(n, sizeof(double)), *hi = (double *)calloc(n, sizeof(double));
+    double *zr = (double *)calloc(n, sizeof(double)), *zi = (double *)calloc(n, sizeof(double));
+    memcpy(hr, h, sizeof(double) * L);
+    memcpy(zr, z, sizeof(double) * L);
+    oracle_fft(hr, hi, n, -1);
+    oracle_fft(zr, zi, n, -1);
+    for (int64_t k = 0; k < n; ++k) {
+        double pr = hr[k] * zr[k] - hi[k] * zi[k];
+        double pi = hr[k] * zi[k] + hi[k] * zr[k];
+        zr[k] = pr; zi[k] = pi;
+    }
+    oracle_fft(zr, zi, n, +1);
+    for (int64_t t = 0; t < L; ++t) out[t] = zr[t] / (double)n;
+    free(hr); free(hi); free(zr); free(zi);
+}
+
+void oracle_causal_conv(const double *h, const double *z, int64_t L, double *out)
+{
+    if (L <= ORACLE_DIRECT_MAX_L) oracle_causal_conv_direct(h, z, L, out);
+    else oracle_causal_conv_fft(h, z, L, out);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Filter spectrum                                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * H[k] = sum_{t<L} h[t] exp(-2 pi i k t / (2L)), k = 0..L: the spectrum of
+ * the filter on the 2L zero-padded grid (bins L+1..2L-1 are the conjugates).
+ * Direct sum for L <= 8192, radix-2 FFT above.
+ */
+void oracle_filter_spectrum(const double *h, int64_t L, double *re, double *im)
+{
+    if (L <= ORACLE_DIRECT_MAX_L) {
+        for (int64_t k = 0; k <= L; ++k) {
+            double ar = 0.0, ai = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                /* reduce k*t mod 2L exactly before forming the angle */
+                int64_t e = (k * t) % (2 * L);
+                double ang = -2.0 * ORACLE_PI * (double)e / (double)(2 * L);
+                ar += h[t] * cos(ang);
+                ai += h[t] * sin(ang);
+            }
+            re[k] = ar; im[k] = ai;
+        }
+        return;
+    }
+    int64_t n = 2 * L;
+    double *xr = (double *)calloc(n, sizeof(double)), *xi = (double *)calloc(n, sizeof(double));
+    memcpy(xr, h, sizeof(double) * L);
+    oracle_fft(xr, xi, n, -1);
+    for (int64_t k = 0; k <= L; ++k) { re[k] = xr[k]; im[k] = xi[k]; }
+    free(xr); free(xi);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Order-N recurrence                                                       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One channel: z_1 = v; z_{n+1}[t] = x_n[t] * (h_n conv z_n)[t]; y = z_{N+1}.
+ * x[n] and h[n] point at the length-L rows of gate n and filter n.
+ */
+void oracle_hyena_channel(const double *v, const double *const *x, const double *const *h,
+                          int64_t L, int N, double *y)
+{
+    double *z = (double *)malloc(sizeof(double) * L);
+    double *c = (double *)malloc(sizeof(double) * L);
+    memcpy(z, v, sizeof(double) * L);
+    for (int n = 0; n < N; ++n) {
+        oracle_causal_conv(h[n], z, L, c);
+        for (int64_t t = 0; t < L; ++t) z[t] = x[n][t] * c[t];
+    }
+    memcpy(y, z, sizeof(double) * L);
+    free(z); free(c);
+}
+
+typedef struct {
+    const double *v, *x, *h;
+    const int *filter_row;   /* per channel: row of h (its channel c) */
+    int64_t L, C;
+    int N, n_filter_rows;
+    double *y;
+    int begin, end;
+} fwd_job;
+
+static void *fwd_worker(void *arg)
+{
+    fwd_job *j = (fwd_job *)arg;
+    const double *xs[64];
+    const double *hs[64];
+    for (int r = j->begin; r < j->end; ++r) {
+        for (int n = 0; n < j->N; ++n) {
+            xs[n] = j->x + ((size_t)n * j->C + r) * j->L;
+            hs[n] = j->h + ((size_t)n * j->n_filter_rows + j->filter_row[r]) * j->L;
+        }
+        oracle_hyena_channel(j->v + (size_t)r * j->L, xs, hs, j->L, j->N, j->y + (size_t)r * j->L);
+    }
+    return NULL;
+}
+
+/*
+ * C independent channels.
+ *   v [C][L], x [N][C][L], h [N][F][L], y [C][L];
+ *   channel r uses filter row filter_row[r] of each h_n (its channel index c).
+ * Work is split over n_threads POSIX threads by channel.
+ */
+int oracle_hyena_forward(const double *v, const double *x, const double *h,
+                         const int *filter_row, int64_t C, int n_filter_rows,
+                         int64_t L, int N, double *y, int n_threads)
+{
+    if (N < 1 || N > 64 || L < 1 || C < 0) return 1;
+    if (C == 0) return 0;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > C) n_threads = (int)C;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n_threads);
+    fwd_job *jobs = (fwd_job *)malloc(sizeof(fwd_job) * n_threads);
+    for (int i = 0; i < n_threads; ++i) {
+        fwd_job j = {v, x, h, filter_row, L, C, N, n_filter_rows, y,
+                     (int)(C * i / n_threads), (int)(C * (i + 1) / n_threads)};
+        jobs[i] = j;
+        pthread_create(&th[i], NULL, fwd_worker, &jobs[i]);
+    }
+    for (int i = 0; i < n_threads; ++i) pthread_join(th[i], NULL);
+    free(th); free(jobs);
+    return 0;
+}
