@@ -1,0 +1,206 @@
+"""Hyena order-N forward on B200 (sm_100a): thin Python binding of libhyena_b200.so.
+
+Every function here marshals arguments (torch CUDA tensors -> device
+pointers, the current CUDA stream) and calls the C ABI declared in
+include/hyena.h; all computation happens in the library's CUDA kernels.
+There is no CPU fallback: if the shared library is missing or a call fails,
+an exception is raised.
+
+    h    = filter_generate(weights, N, D, L, alpha_lo, alpha_hi)      # [N][D][L] fp32
+    hhat = [filter_rfft(h[n]) for n in range(N)]                      # cached spectra
+    y    = forward(v, [x1, ..., xN], hhat)                            # [B][D][L]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libhyena_b200.so")
+
+HYENA_OK, HYENA_ERR_INVALID_ARG, HYENA_ERR_UNSUPPORTED, HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA = range(5)
+HYENA_F32, HYENA_BF16 = 0, 1
+
+# exported symbols (kept in step with include/hyena.h)
+EXPORTS = (
+    "hyena_filter_generate", "hyena_filter_spectrum_bytes", "hyena_filter_rfft", "hyena_spectrum_layout",
+    "hyena_forward_workspace_bytes", "hyena_forward", "hyena_status_string", "hyena_last_cuda_error",
+    "hyena_abi_version",
+)
+
+
+class HyenaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = load()
+        msg = lib.hyena_status_string(status).decode()
+        if status == HYENA_ERR_CUDA:
+            msg += ": " + lib.hyena_last_cuda_error().decode()
+        super().__init__(f"{where}: {msg}")
+        self.status = status
+
+
+class FilterParams(ctypes.Structure):
+    _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+                ("b2", ctypes.c_void_p), ("W3", ctypes.c_void_p), ("b3", ctypes.c_void_p),
+                ("n_bands", ctypes.c_int), ("width", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libhyena_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m fft_long_convolution_implicit_b200.build`")
+    l = ctypes.CDLL(LIB_PATH)
+    i, sz, P = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    l.hyena_filter_generate.argtypes = [ctypes.POINTER(FilterParams), i, i, i, ctypes.c_float, ctypes.c_float, P, P]
+    l.hyena_filter_generate.restype = i
+    l.hyena_filter_spectrum_bytes.argtypes = [i, i]
+    l.hyena_filter_spectrum_bytes.restype = sz
+    l.hyena_filter_rfft.argtypes = [P, i, i, P, P]
+    l.hyena_filter_rfft.restype = i
+    l.hyena_spectrum_layout.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i)]
+    l.hyena_spectrum_layout.restype = i
+    l.hyena_forward_workspace_bytes.argtypes = [i, i, i, i, i]
+    l.hyena_forward_workspace_bytes.restype = sz
+    l.hyena_forward.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
+    l.hyena_forward.restype = i
+    l.hyena_status_string.argtypes = [i]
+    l.hyena_status_string.restype = ctypes.c_char_p
+    l.hyena_last_cuda_error.argtypes = []
+    l.hyena_last_cuda_error.restype = ctypes.c_char_p
+    l.hyena_abi_version.argtypes = []
+    l.hyena_abi_version.restype = i
+    _lib = l
+    return l
+
+
+def _check(status: int, where: str):
+    if status != HYENA_OK:
+        raise HyenaError(status, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return HYENA_F32
+    if t.dtype == torch.bfloat16:
+        return HYENA_BF16
+    raise TypeError(f"unsupported activation dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t, name):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# ------------------------------------------------------------------ queries --
+
+def abi_version() -> int:
+    return load().hyena_abi_version()
+
+
+def filter_spectrum_bytes(D: int, L: int) -> int:
+    return load().hyena_filter_spectrum_bytes(D, L)
+
+
+def forward_workspace_bytes(B: int, D: int, L: int, N: int, bf16: bool) -> int:
+    return load().hyena_forward_workspace_bytes(B, D, L, N, HYENA_BF16 if bf16 else HYENA_F32)
+
+
+def spectrum_layout(L: int) -> tuple[int, int, int]:
+    """(M, M1, MV): bin k < M of channel c sits at float2 index c*M + (k % M1)*MV + k // M1."""
+    M, M1, MV = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(load().hyena_spectrum_layout(L, ctypes.byref(M), ctypes.byref(M1), ctypes.byref(MV)),
+           "hyena_spectrum_layout")
+    return M.value, M1.value, MV.value
+
+
+# ------------------------------------------------------------------- calls --
+
+def filter_generate(weights: dict, N: int, D: int, L: int, alpha_lo: float, alpha_hi: float,
+                    h=None, n_bands: int = 8, stream=None):
+    """Implicit filters h [N][D][L] (float32) from FFN weights (CUDA float32
+    tensors W1 [H][1+2K], b1, W2 [H][H], b2, W3 [N*D][H], b3)."""
+    torch = _torch()
+    W1 = weights["W1"]
+    dev = W1.device
+    if h is None:
+        h = torch.empty((N, D, L), dtype=torch.float32, device=dev)
+    p = FilterParams(*(ctypes.c_void_p(_dev(weights[k], k).value) for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
+                     n_bands, W1.shape[0])
+    _check(load().hyena_filter_generate(ctypes.byref(p), N, D, L, alpha_lo, alpha_hi, _dev(h, "h"),
+                                        _stream(stream)), "hyena_filter_generate")
+    return h
+
+
+def filter_rfft(h, hhat=None, stream=None):
+    """Spectrum block (uint8 CUDA tensor, library order) of one filter h [D][L] float32."""
+    torch = _torch()
+    D, L = h.shape
+    nbytes = filter_spectrum_bytes(D, L)
+    if nbytes == 0:
+        _check(HYENA_ERR_UNSUPPORTED, "hyena_filter_spectrum_bytes")
+    if hhat is None:
+        hhat = torch.empty(nbytes, dtype=torch.uint8, device=h.device)
+    _check(load().hyena_filter_rfft(_dev(h, "h"), D, L, _dev(hhat, "hhat"), _stream(stream)), "hyena_filter_rfft")
+    return hhat
+
+
+def forward(v, xs, hhats, y=None, workspace=None, stream=None):
+    """y = z_{N+1} of the order-N recurrence for v, gates xs[0..N-1] ([B][D][L],
+    float32 or bfloat16) and cached spectra hhats[0..N-1]."""
+    torch = _torch()
+    B, D, L = v.shape
+    N = len(xs)
+    if len(hhats) != N:
+        raise ValueError("need one spectrum per gate")
+    code = _dtype_code(v)
+    for x in xs:
+        if x.shape != v.shape or x.dtype != v.dtype:
+            raise ValueError("gates must match v in shape and dtype")
+    if y is None:
+        y = torch.empty_like(v)
+    ws_need = forward_workspace_bytes(B, D, L, N, code == HYENA_BF16)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=v.device)
+    xarr = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+    harr = (ctypes.c_void_p * N)(*[_dev(hh, "hhat").value for hh in hhats])
+    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().hyena_forward(_dev(v, "v"), xarr, harr, B, D, L, N, code, _dev(y, "y"), ws_ptr, ws_bytes,
+                                _stream(stream)), "hyena_forward")
+    return y
+
+
+def spectrum_natural(hhat, D: int, L: int):
+    """View a spectrum block in natural bin order: complex [D][M+1] (torch,
+    on the block's device), M = max(L, 128). Index permutation only."""
+    torch = _torch()
+    M, M1, MV = spectrum_layout(L)
+    blk = hhat[: D * M * 8].view(torch.float32).view(D, M, 2)
+    k = torch.arange(M, device=hhat.device)
+    idx = (k % M1) * MV + k // M1
+    nat = blk[:, idx, :]
+    out = torch.complex(nat[..., 0], nat[..., 1])
+    out = torch.cat([out, torch.zeros(D, 1, dtype=out.dtype, device=out.device)], dim=1)
+    out[:, M] = blk[:, 0, 1].to(out.dtype)       # packed Nyquist bin
+    out[:, 0] = blk[:, 0, 0].to(out.dtype)
+    return out

@@ -1,0 +1,208 @@
+// api.cu -- C ABI: argument checks, layout, dispatch to the kernels.
+#include <mutex>
+#include <unordered_map>
+
+#include "hyena.h"
+#include "kernels.cuh"
+
+using namespace hyena;
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+
+hyena_status cuda_fail(cudaError_t e) {
+  const char* s = cudaGetErrorString(e);
+  size_t i = 0;
+  for (; s && s[i] && i + 1 < sizeof(g_last_cuda_error); ++i) g_last_cuda_error[i] = s[i];
+  g_last_cuda_error[i] = 0;
+  return HYENA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return p && ((reinterpret_cast<uintptr_t>(p) & 15u) == 0); }
+
+// L2-sized wave of four-step channels
+constexpr size_t kWaveTargetBytes = size_t(48) << 20;
+constexpr long long kMaxGridY = 65535;
+
+struct GridKey {
+  const void* k;
+  int dev;
+  int threads;
+  size_t smem;
+  bool operator==(const GridKey& o) const { return k == o.k && dev == o.dev && threads == o.threads && smem == o.smem; }
+};
+struct GridKeyHash {
+  size_t operator()(const GridKey& g) const {
+    return std::hash<const void*>()(g.k) ^ (size_t(g.dev) << 48) ^ (size_t(g.threads) << 32) ^ g.smem;
+  }
+};
+std::mutex g_grid_mu;
+std::unordered_map<GridKey, int, GridKeyHash> g_grid_cache;
+
+}  // namespace
+
+cudaError_t hyena::persistent_grid(const void* kernel, int threads, size_t smem, int* grid) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  GridKey key{kernel, dev, threads, smem};
+  {
+    std::lock_guard<std::mutex> lk(g_grid_mu);
+    auto it = g_grid_cache.find(key);
+    if (it != g_grid_cache.end()) {
+      *grid = it->second;
+      return cudaSuccess;
+    }
+  }
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  *grid = sms * per_sm;
+  std::lock_guard<std::mutex> lk(g_grid_mu);
+  g_grid_cache[key] = *grid;
+  return cudaSuccess;
+}
+
+extern "C" {
+
+int hyena_abi_version(void) { return HYENA_ABI_VERSION; }
+
+const char* hyena_status_string(hyena_status s) {
+  switch (s) {
+    case HYENA_OK: return "ok";
+    case HYENA_ERR_INVALID_ARG: return "invalid argument";
+    case HYENA_ERR_UNSUPPORTED: return "unsupported length (L must be a power of two in [16, 2^20])";
+    case HYENA_ERR_WORKSPACE: return "workspace missing or too small";
+    case HYENA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* hyena_last_cuda_error(void) { return g_last_cuda_error; }
+
+hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {
+  Layout y;
+  if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
+  if (M) *M = y.M;
+  if (M1) *M1 = y.M1;
+  if (MV) *MV = y.MV;
+  return HYENA_OK;
+}
+
+size_t hyena_filter_spectrum_bytes(int D, int L) {
+  Layout y;
+  if (D < 1 || !make_layout(L, &y)) return 0;
+  return sizeof(float2) * spectrum_block_floats2(y, D);
+}
+
+hyena_status hyena_filter_generate(const hyena_filter_params* p, int N, int D, int L, float alpha_lo,
+                                   float alpha_hi, float* h, hyena_stream stream) {
+  if (!p || !h || N < 1 || N > kMaxOrder || D < 1) return HYENA_ERR_INVALID_ARG;
+  if (!p->W1 || !p->b1 || !p->W2 || !p->b2 || !p->W3 || !p->b3) return HYENA_ERR_INVALID_ARG;
+  if (p->n_bands < 1 || p->n_bands > 32 || p->width < 1 || p->width > 128) return HYENA_ERR_INVALID_ARG;
+  if (!aligned16(h)) return HYENA_ERR_INVALID_ARG;
+  if ((long long)N * D > (1LL << 30)) return HYENA_ERR_INVALID_ARG;
+  Layout y;
+  if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_filter_generate(p->W1, p->b1, p->W2, p->b2, p->W3, p->b3, p->n_bands, p->width, N, D, L,
+                                         alpha_lo, alpha_hi, h, (cudaStream_t)stream);
+  return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
+}
+
+hyena_status hyena_filter_rfft(const float* h, int D, int L, void* hhat, hyena_stream stream) {
+  if (!aligned16(h) || !aligned16(hhat) || D < 1) return HYENA_ERR_INVALID_ARG;
+  Layout y;
+  if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  float2* spec = reinterpret_cast<float2*>(hhat);
+  float2* tables = spec + (size_t)D * y.M;
+  cudaError_t e = launch_fill_tables(tables, y, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (!y.fourstep) {
+    e = launch_fused_spectrum(h, spec, tables, D, L, y.logMV, s);
+  } else {
+    for (long long c0 = 0; c0 < D && e == cudaSuccess; c0 += kMaxGridY) {
+      const int nd = (int)((D - c0) < kMaxGridY ? (D - c0) : kMaxGridY);
+      e = launch_fourstep_spectrum(h + (size_t)c0 * L, spec + (size_t)c0 * y.M, tables, nd, y, s);
+    }
+  }
+  return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
+}
+
+size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dtype) {
+  Layout y;
+  if (B < 1 || D < 1 || N < 1 || N > kMaxOrder || (dtype != HYENA_F32 && dtype != HYENA_BF16)) return 0;
+  if (!make_layout(L, &y)) return 0;
+  if (!y.fourstep) return 0;
+  const size_t per = sizeof(float2) * (size_t)y.M;
+  long long w = (long long)(kWaveTargetBytes / per);
+  if (w < 1) w = 1;
+  const long long C = (long long)B * D;
+  if (w > C) w = C;
+  if (w > kMaxGridY) w = kMaxGridY;
+  return per * (size_t)w;
+}
+
+hyena_status hyena_forward(const void* v, const void* const* x, const void* const* hhat, int B, int D, int L,
+                           int N, hyena_dtype dtype, void* y, void* workspace, size_t workspace_bytes,
+                           hyena_stream stream) {
+  if (N < 1 || N > kMaxOrder || B < 1 || D < 1) return HYENA_ERR_INVALID_ARG;
+  if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+  if (!x || !hhat || !aligned16(v) || !aligned16(y)) return HYENA_ERR_INVALID_ARG;
+  for (int n = 0; n < N; ++n)
+    if (!aligned16(x[n]) || !aligned16(hhat[n])) return HYENA_ERR_INVALID_ARG;
+  if ((long long)B * D > (1LL << 40) / (L > 0 ? L : 1)) return HYENA_ERR_INVALID_ARG;
+  Layout ly;
+  if (!make_layout(L, &ly)) return HYENA_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + (size_t)D * ly.M;
+  cudaError_t e = cudaSuccess;
+  if (!ly.fourstep) {
+    FusedLaunch p{};
+    p.v = v;
+    for (int n = 0; n < N; ++n) {
+      p.x[n] = x[n];
+      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
+    }
+    p.y = y;
+    p.tables = tables;
+    p.B = B; p.D = D; p.L = L; p.N = N;
+    p.bf16 = (dtype == HYENA_BF16);
+    e = launch_fused_forward(p, ly.logMV, s);
+  } else {
+    const size_t per = sizeof(float2) * (size_t)ly.M;
+    if (!aligned16(workspace) || workspace_bytes < per) return HYENA_ERR_WORKSPACE;
+    const long long C = (long long)B * D;
+    long long w = (long long)(workspace_bytes / per);
+    if (w > C) w = C;
+    if (w > kMaxGridY) w = kMaxGridY;
+    FourStepLaunch p{};
+    p.v = v;
+    for (int n = 0; n < N; ++n) {
+      p.x[n] = x[n];
+      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
+    }
+    p.y = y;
+    p.tables = tables;
+    p.scratch = reinterpret_cast<float2*>(workspace);
+    p.B = B; p.D = D; p.L = L; p.N = N;
+    p.bf16 = (dtype == HYENA_BF16);
+    for (long long c0 = 0; c0 < C && e == cudaSuccess; c0 += w) {
+      p.ch0 = c0;
+      p.wave = (int)((C - c0) < w ? (C - c0) : w);
+      e = launch_fourstep_wave(p, ly, s);
+    }
+  }
+  return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
+}
+
+}  // extern "C"

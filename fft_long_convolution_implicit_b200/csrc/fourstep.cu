@@ -1,0 +1,323 @@
+// fourstep.cu -- Hyena order-N forward for 8192 < L <= 2^20.
+//
+// The packed M-point transform (M = L) is split M = M1 * MV, input index
+// m = MV n1 + n2, output bin k = k1 + M1 k2:
+//   column pass: M1-point DFTs over n1 for each n2  -> A[k1][n2]
+//   row pass:    twiddle w_M^{n2 k1}, MV-point FFT over n2 -> bins k1 + M1 k2;
+//                rows k1 and M1-k1 hold mirror bins, so one CTA takes both,
+//                forms the spectral product and runs the inverse row FFT and
+//                conjugate twiddle in place             -> E[k1][n2]
+//   column pass: inverse M1-point DFTs over k1, keep n1 < M1/2 (first L real
+//                outputs), gate with x_n, and -- between stages -- the next
+//                stage's forward column DFTs on the same column.
+// A channel's A/E array lives in a caller workspace and is visited by
+// 2N + 1 launches per wave of channels; waves are sized by the workspace so
+// that the array stays resident in L2.
+#include "kernels.cuh"
+#include "paired.cuh"
+
+namespace hyena {
+
+enum ColMode { kColFirst = 0, kColMid = 1, kColLast = 2, kColSpecFirst = 3 };
+
+template <int MB>
+struct ColCfg {
+  static constexpr int M1 = 16 * MB;
+  static constexpr int CW = MB == 1 ? 128 : (MB == 2 ? 64 : 32);   // columns per CTA
+  static constexpr int THREADS = CW * MB;
+  static constexpr int VEC = padded_len(M1) + 1;                  // smem stride of one column
+  static constexpr size_t SMEM = MB == 1 ? 0 : sizeof(float2) * (size_t)CW * VEC;
+};
+
+// exp(-2 pi i e / M) for an integer exponent e in [0, M)
+__device__ __forceinline__ float2 expi_neg(int e, int M) {
+  float s, c;
+  sincospif(2.0f * (float)e / (float)M, &s, &c);
+  return make_float2(c, -s);
+}
+
+// Column pass. Thread (j, col): column n2 = tile*CW + col; in the 16-point
+// stage it owns rows n1 = j + r*MB; in the MB-point stage butterflies
+// jj = j + q*MB (bins jj + 16 r).
+template <int MB, int MODE, typename T>
+__global__ void __launch_bounds__(ColCfg<MB>::THREADS)
+col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict__ yout, float2* __restrict__ scr,
+           const float2* __restrict__ tw1, int B, int D, int L, int MV, long long ch0) {
+  using Cfg = ColCfg<MB>;
+  constexpr int M1 = Cfg::M1, CW = Cfg::CW, NQ = 16 / MB;
+  extern __shared__ float2 sm[];
+  const int tid = threadIdx.x;
+  const int col = tid % CW, j = tid / CW;
+  const int n2 = blockIdx.x * CW + col;
+  const long long ch = ch0 + blockIdx.y;
+  const int c = (int)(ch / B), b = (int)(ch % B);
+  const size_t row = ((size_t)b * D + c) * (size_t)L;
+  float2* __restrict__ S = scr + (size_t)blockIdx.y * ((size_t)M1 * MV);
+  float2* csm = sm + col * Cfg::VEC;
+  float2 a[16];
+
+  if constexpr (MODE == kColFirst || MODE == kColSpecFirst) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const size_t m = (size_t)MV * (j + r * MB) + n2;
+      a[r] = IO<T>::load2_stream(zin + row + 2 * m);
+    }
+  } else {
+    if constexpr (MB == 1) {
+#pragma unroll
+      for (int r = 0; r < 16; ++r) a[r] = S[(size_t)r * MV + n2];
+    } else {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int r = 0; r < MB; ++r) a[q * MB + r] = S[(size_t)(j + q * MB + 16 * r) * MV + n2];
+      dft_blocks<MB, true>(a);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int jj = j + q * MB;
+#pragma unroll
+        for (int r = 1; r < MB; ++r) a[q * MB + r] = cmulc(a[q * MB + r], __ldg(&tw1[15 + (r - 1) * 16 + jj]));
+#pragma unroll
+        for (int r = 0; r < MB; ++r) csm[pidx(jj + 16 * r)] = a[q * MB + r];
+      }
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < 16; ++r) a[r] = csm[pidx(16 * j + r)];
+    }
+    dft16<true, false, true, 0>(a);          // outputs n1 = j + r*MB, r < 8
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const size_t m = (size_t)MV * (j + r * MB) + n2;
+      const float2 g = IO<T>::load2_stream(gate + row + 2 * m);
+      a[r] = make_float2(a[r].x * g.x, a[r].y * g.y);
+    }
+    if constexpr (MODE == kColLast) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const size_t m = (size_t)MV * (j + r * MB) + n2;
+        IO<T>::store2(yout + row + 2 * m, a[r]);
+      }
+      return;
+    }
+  }
+  // forward column transform (upper half of the column is zero)
+  dft16<false, true, false, 0>(a);
+  if constexpr (MB == 1) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) S[(size_t)r * MV + n2] = a[r];
+  } else {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) csm[pidx(16 * j + r)] = a[r];
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int jj = j + q * MB;
+#pragma unroll
+      for (int r = 0; r < MB; ++r) a[q * MB + r] = csm[pidx(jj + 16 * r)];
+#pragma unroll
+      for (int r = 1; r < MB; ++r) a[q * MB + r] = cmul(a[q * MB + r], __ldg(&tw1[15 + (r - 1) * 16 + jj]));
+    }
+    dft_blocks<MB, false>(a);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int r = 0; r < MB; ++r) S[(size_t)(j + q * MB + 16 * r) * MV + n2] = a[q * MB + r];
+  }
+}
+
+// Row pass on rows kA and kB (kA + kB = M1, or the self-mirrored rows 0 and
+// M1/2 in CTA 0). Threads [0, TV) work on row kA, [TV, 2 TV) on row kB.
+template <int LOGMV, int MODE>
+__global__ void __launch_bounds__(2 * Plan<LOGMV>::TV)
+row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const float2* __restrict__ tables, int M1,
+           int B, long long ch0) {
+  using P = Plan<LOGMV>;
+  constexpr int MV = P::MV, TV = P::TV, Q8 = MV / 8, Q16 = MV / 16, VEC = padded_len(MV);
+  extern __shared__ float2 sm[];
+  const int M = M1 * MV;
+  const float2* __restrict__ tw = tables;
+  const float2* __restrict__ Wv = tables + MV;
+  const int p = blockIdx.x;
+  const int kA = p, kB = (p == 0) ? M1 / 2 : M1 - p;
+  float2* S;
+  float2* H;
+  if (MODE == kPairConv) {
+    S = scr + (size_t)blockIdx.y * M;
+    const long long ch = ch0 + blockIdx.y;
+    H = const_cast<float2*>(spec) + (size_t)(ch / B) * M;
+  } else {
+    S = scr + (size_t)blockIdx.y * M;   // spectrum block of channel blockIdx.y, transformed in place
+    H = S;
+  }
+  const int t = threadIdx.x;
+  const int vec = t / TV, tl = t % TV;
+  const int krow = vec ? kB : kA;
+  float2* base = sm + vec * VEC;
+  float2* src = S + (size_t)krow * MV;
+
+  // four-step twiddle w_M^{krow n2}, n2 = tl + r*Q16
+  const float2 tw0 = expi_neg((int)(((long long)krow * tl) % M), M);
+  const float2 tstep = expi_neg((int)(((long long)krow * Q16) % M), M);
+  float2 a[16];
+#pragma unroll
+  for (int r = 0; r < 16; ++r) a[r] = src[tl + r * Q16];
+  {
+    float2 cur = tw0;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      a[r] = cmul(a[r], cur);
+      cur = cmul(cur, tstep);
+    }
+  }
+  dft16<false, false, false, 0>(a);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) base[pidx(16 * tl + r)] = a[r];
+  __syncthreads();
+  mid_fwd_all<LOGMV>(a, base, tw, tl);
+
+  {
+    float2 *bA, *bB, *HA, *HB;
+    int jA, jB;
+    bool head = false, has_rho = true;
+    float2 rho;
+    if (p != 0) {
+      bA = sm; bB = sm + VEC;
+      jA = t; jB = Q8 - 1 - t;
+      float s, c;
+      sincospif((float)kA / (float)M, &s, &c);
+      rho = make_float2(c, -s);
+      HA = H + (size_t)kA * MV; HB = H + (size_t)kB * MV;
+    } else if (t < Q16) {
+      bA = bB = sm;
+      head = (t == 0);
+      jA = head ? 0 : t; jB = head ? Q16 : Q8 - t;
+      rho = make_float2(1.f, 0.f); has_rho = false;
+      HA = HB = H;
+    } else {
+      const int t2 = t - Q16;
+      bA = bB = sm + VEC;
+      jA = t2; jB = Q8 - 1 - t2;
+      float s, c;
+      sincospif((float)(M1 / 2) / (float)M, &s, &c);
+      rho = make_float2(c, -s);
+      HA = HB = H + (size_t)(M1 / 2) * MV;
+    }
+    paired_pass<LOGMV, MODE>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
+  }
+  if (MODE == kPairSpectrum) return;
+  __syncthreads();
+  mid_inv_all<LOGMV>(a, base, tw, tl);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) a[r] = base[pidx(16 * tl + r)];
+  dft16<true, false, false, 0>(a);
+  {
+    float2 cur = tw0;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      a[r] = cmulc(a[r], cur);
+      cur = cmul(cur, tstep);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 16; ++r) src[tl + r * Q16] = a[r];
+}
+
+// ------------------------------------------------------------- launchers --
+
+template <typename K>
+static cudaError_t prep(K kernel, size_t smem) {
+  if (smem > 48 * 1024) return cudaFuncSetAttribute((const void*)kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  return cudaSuccess;
+}
+
+template <int MB, int MODE, typename T>
+static cudaError_t launch_col(const T* zin, const T* gate, T* yout, float2* scr, const float2* tw1, int B, int D,
+                              int L, int MV, long long ch0, int nch, cudaStream_t s) {
+  using Cfg = ColCfg<MB>;
+  auto k = col_kernel<MB, MODE, T>;
+  cudaError_t e = prep(k, Cfg::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(MV / Cfg::CW, nch);
+  k<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(zin, gate, yout, scr, tw1, B, D, L, MV, ch0);
+  return cudaGetLastError();
+}
+
+template <int LOGMV, int MODE>
+static cudaError_t launch_row(float2* scr, const float2* spec, const float2* tables, int M1, int B, long long ch0,
+                              int nch, cudaStream_t s) {
+  auto k = row_kernel<LOGMV, MODE>;
+  const size_t smem = sizeof(float2) * 2 * (size_t)padded_len(1 << LOGMV);
+  cudaError_t e = prep(k, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(M1 / 2, nch);
+  k<<<grid, 2 * Plan<LOGMV>::TV, smem, s>>>(scr, spec, tables, M1, B, ch0);
+  return cudaGetLastError();
+}
+
+template <int LOGMV, int MB, typename T>
+static cudaError_t wave_t(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
+  const float2* tw1 = p.tables + y.tw_1;
+  const int MV = y.MV;
+  cudaError_t e = launch_col<MB, kColFirst, T>(reinterpret_cast<const T*>(p.v), nullptr, nullptr, p.scratch, tw1,
+                                               p.B, p.D, p.L, MV, p.ch0, p.wave, s);
+  for (int n = 0; n < p.N && e == cudaSuccess; ++n) {
+    e = launch_row<LOGMV, kPairConv>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);
+    if (e != cudaSuccess) break;
+    const T* g = reinterpret_cast<const T*>(p.x[n]);
+    if (n + 1 < p.N)
+      e = launch_col<MB, kColMid, T>(nullptr, g, nullptr, p.scratch, tw1, p.B, p.D, p.L, MV, p.ch0, p.wave, s);
+    else
+      e = launch_col<MB, kColLast, T>(nullptr, g, reinterpret_cast<T*>(p.y), p.scratch, tw1, p.B, p.D, p.L, MV,
+                                      p.ch0, p.wave, s);
+  }
+  return e;
+}
+
+template <int LOGMV, int MB>
+static cudaError_t wave_lm(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
+  return p.bf16 ? wave_t<LOGMV, MB, __nv_bfloat16>(p, y, s) : wave_t<LOGMV, MB, float>(p, y, s);
+}
+
+cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
+  if (y.logMV == 10 && y.mb == 1) return wave_lm<10, 1>(p, y, s);
+  if (y.logMV == 11 && y.mb == 1) return wave_lm<11, 1>(p, y, s);
+  if (y.logMV == 12) {
+    switch (y.mb) {
+      case 1: return wave_lm<12, 1>(p, y, s);
+      case 2: return wave_lm<12, 2>(p, y, s);
+      case 4: return wave_lm<12, 4>(p, y, s);
+      case 8: return wave_lm<12, 8>(p, y, s);
+      case 16: return wave_lm<12, 16>(p, y, s);
+      default: break;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int LOGMV, int MB>
+static cudaError_t spec_lm(const float* h, float2* spec, const float2* tables, int D, const Layout& y,
+                           cudaStream_t s) {
+  cudaError_t e = launch_col<MB, kColSpecFirst, float>(h, nullptr, nullptr, spec, tables + y.tw_1, 1, D, y.L, y.MV,
+                                                       0, D, s);
+  if (e != cudaSuccess) return e;
+  return launch_row<LOGMV, kPairSpectrum>(spec, spec, tables, y.M1, 1, 0, D, s);
+}
+
+cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D, const Layout& y,
+                                     cudaStream_t s) {
+  if (y.logMV == 10 && y.mb == 1) return spec_lm<10, 1>(h, spec, tables, D, y, s);
+  if (y.logMV == 11 && y.mb == 1) return spec_lm<11, 1>(h, spec, tables, D, y, s);
+  if (y.logMV == 12) {
+    switch (y.mb) {
+      case 1: return spec_lm<12, 1>(h, spec, tables, D, y, s);
+      case 2: return spec_lm<12, 2>(h, spec, tables, D, y, s);
+      case 4: return spec_lm<12, 4>(h, spec, tables, D, y, s);
+      case 8: return spec_lm<12, 8>(h, spec, tables, D, y, s);
+      case 16: return spec_lm<12, 16>(h, spec, tables, D, y, s);
+      default: break;
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace hyena

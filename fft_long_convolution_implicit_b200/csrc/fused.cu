@@ -1,0 +1,175 @@
+// fused.cu -- Hyena order-N forward for L <= 8192: one CTA per channel at a
+// time (persistent over channels), z resident in shared memory across all N
+// stages. HBM sees v, x_1..x_N and the filter spectra once and y once.
+//
+// Stage n (order-N recurrence, "Hyena Hierarchy" digest, 방법 / 프레임워크
+// 개요; explainer "Hyena 演算子の形"):
+//   z_{n+1} = x_n * (h_n conv z_n), conv = causal, via the 2L-grid FFT.
+// Thread tl holds packed points m = tl + r*M/16 (r < 8) of z between stages:
+// these are exactly the inputs of the first forward pass and the outputs of
+// the last inverse pass, so the gate and the stage hand-off stay in registers.
+#include "kernels.cuh"
+#include "paired.cuh"
+
+namespace hyena {
+
+template <int LOGMV, typename T>
+__global__ void __launch_bounds__(Plan<LOGMV>::TV)
+fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __restrict__ y,
+                     const float2* __restrict__ tables, int B, int D, int L, int N) {
+  using P = Plan<LOGMV>;
+  constexpr int MV = P::MV, Q8 = MV / 8, Q16 = MV / 16;
+  extern __shared__ float2 sm[];
+  const int tl = threadIdx.x;
+  const float2* __restrict__ tw = tables;
+  const float2* __restrict__ Wv = tables + MV;
+  const long long C = (long long)B * D;
+  const bool head = (tl == 0);
+  const int jA = head ? 0 : tl;
+  const int jB = head ? Q16 : Q8 - tl;
+  const float2 one = make_float2(1.f, 0.f);
+
+  for (long long ch = blockIdx.x; ch < C; ch += gridDim.x) {
+    // channel order c-major so that CTAs sharing a filter run side by side
+    const int c = (int)(ch / B), b = (int)(ch % B);
+    const size_t row = ((size_t)b * D + c) * (size_t)L;
+    float2 a[16];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int m = tl + r * Q16;
+      a[r] = (2 * m < L) ? IO<T>::load2_stream(v + row + 2 * m) : make_float2(0.f, 0.f);
+    }
+    for (int n = 0; n < N; ++n) {
+      // forward: first pass (radix 16, upper half of the input is zero)
+      dft16<false, true, false, 0>(a);
+#pragma unroll
+      for (int r = 0; r < 16; ++r) sm[pidx(16 * tl + r)] = a[r];
+      __syncthreads();
+      mid_fwd_all<LOGMV>(a, sm, tw, tl);
+      // last forward pass + spectral product + first inverse pass
+      float2* H = const_cast<float2*>(pick(hh, n)) + (size_t)c * MV;
+      paired_pass<LOGMV, kPairConv>(sm, sm, jA, jB, head, tw, Wv, one, false, H, H, 0.f);
+      __syncthreads();
+      mid_inv_all<LOGMV>(a, sm, tw, tl);
+      // last inverse pass (radix 16): only the first half of the outputs is kept
+#pragma unroll
+      for (int r = 0; r < 16; ++r) a[r] = sm[pidx(16 * tl + r)];
+      dft16<true, false, true, 0>(a);
+      // gate: z_{n+1}[t] = x_n[t] * conv[t]
+      const T* __restrict__ xr = pick(x, n) + row;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int m = tl + r * Q16;
+        const float2 g = (2 * m < L) ? IO<T>::load2_stream(xr + 2 * m) : make_float2(0.f, 0.f);
+        a[r] = make_float2(a[r].x * g.x, a[r].y * g.y);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int m = tl + r * Q16;
+      if (2 * m < L) IO<T>::store2(y + row + 2 * m, a[r]);
+    }
+  }
+}
+
+// Filter spectrum for the fused layout: H[c][k] = rfft(pad(h_c, 2M))[k] / (4M)
+// in natural order k < M, bin 0 holding (H[0], H[M]) (both real).
+template <int LOGMV>
+__global__ void __launch_bounds__(Plan<LOGMV>::TV)
+fused_spectrum_kernel(const float* __restrict__ h, float2* __restrict__ spec, const float2* __restrict__ tables,
+                      int D, int L) {
+  using P = Plan<LOGMV>;
+  constexpr int MV = P::MV, Q8 = MV / 8, Q16 = MV / 16;
+  extern __shared__ float2 sm[];
+  const int tl = threadIdx.x;
+  const float2* __restrict__ tw = tables;
+  const float2* __restrict__ Wv = tables + MV;
+  const bool head = (tl == 0);
+  const int jA = head ? 0 : tl;
+  const int jB = head ? Q16 : Q8 - tl;
+  const float scale = 1.0f / (8.0f * (float)MV);
+  for (int c = blockIdx.x; c < D; c += gridDim.x) {
+    const float* __restrict__ hr = h + (size_t)c * L;
+    float2 a[16];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int m = tl + r * Q16;
+      a[r] = (2 * m < L) ? __ldg(reinterpret_cast<const float2*>(hr + 2 * m)) : make_float2(0.f, 0.f);
+    }
+    dft16<false, true, false, 0>(a);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) sm[pidx(16 * tl + r)] = a[r];
+    __syncthreads();
+    mid_fwd_all<LOGMV>(a, sm, tw, tl);
+    float2* H = spec + (size_t)c * MV;
+    paired_pass<LOGMV, kPairSpectrum>(sm, sm, jA, jB, head, tw, Wv, make_float2(1.f, 0.f), false, H, H, scale);
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------- launchers --
+
+template <int LOGMV, typename T>
+static cudaError_t launch_fused_t(const FusedLaunch& p, cudaStream_t s) {
+  auto k = fused_forward_kernel<LOGMV, T>;
+  const int threads = Plan<LOGMV>::TV;
+  const size_t smem = sizeof(float2) * padded_len(1 << LOGMV);
+  int grid = 0;
+  cudaError_t e = persistent_grid((const void*)k, threads, smem, &grid);
+  if (e != cudaSuccess) return e;
+  long long C = (long long)p.B * p.D;
+  if ((long long)grid > C) grid = (int)C;
+  GatePtrs<T> xp;
+  for (int i = 0; i < kMaxOrder; ++i) xp.p[i] = reinterpret_cast<const T*>(p.x[i]);
+  k<<<grid, threads, smem, s>>>(reinterpret_cast<const T*>(p.v), xp, p.hh, reinterpret_cast<T*>(p.y),
+                                p.tables, p.B, p.D, p.L, p.N);
+  return cudaGetLastError();
+}
+
+template <int LOGMV>
+static cudaError_t launch_fused_l(const FusedLaunch& p, cudaStream_t s) {
+  return p.bf16 ? launch_fused_t<LOGMV, __nv_bfloat16>(p, s) : launch_fused_t<LOGMV, float>(p, s);
+}
+
+cudaError_t launch_fused_forward(const FusedLaunch& p, int logMV, cudaStream_t s) {
+  switch (logMV) {
+    case 7: return launch_fused_l<7>(p, s);
+    case 8: return launch_fused_l<8>(p, s);
+    case 9: return launch_fused_l<9>(p, s);
+    case 10: return launch_fused_l<10>(p, s);
+    case 11: return launch_fused_l<11>(p, s);
+    case 12: return launch_fused_l<12>(p, s);
+    case 13: return launch_fused_l<13>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int LOGMV>
+static cudaError_t launch_fused_spec_l(const float* h, float2* spec, const float2* tables, int D, int L,
+                                       cudaStream_t s) {
+  auto k = fused_spectrum_kernel<LOGMV>;
+  const int threads = Plan<LOGMV>::TV;
+  const size_t smem = sizeof(float2) * padded_len(1 << LOGMV);
+  int grid = 0;
+  cudaError_t e = persistent_grid((const void*)k, threads, smem, &grid);
+  if (e != cudaSuccess) return e;
+  if (grid > D) grid = D;
+  k<<<grid, threads, smem, s>>>(h, spec, tables, D, L);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* tables, int D, int L, int logMV,
+                                  cudaStream_t s) {
+  switch (logMV) {
+    case 7: return launch_fused_spec_l<7>(h, spec, tables, D, L, s);
+    case 8: return launch_fused_spec_l<8>(h, spec, tables, D, L, s);
+    case 9: return launch_fused_spec_l<9>(h, spec, tables, D, L, s);
+    case 10: return launch_fused_spec_l<10>(h, spec, tables, D, L, s);
+    case 11: return launch_fused_spec_l<11>(h, spec, tables, D, L, s);
+    case 12: return launch_fused_spec_l<12>(h, spec, tables, D, L, s);
+    case 13: return launch_fused_spec_l<13>(h, spec, tables, D, L, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace hyena

@@ -1,0 +1,71 @@
+// kernels.cuh -- launch parameter structs and launcher prototypes shared by
+// the host dispatch (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "layout.h"
+
+namespace hyena {
+
+constexpr int kMaxOrder = 8;
+
+template <typename T>
+struct GatePtrs {
+  const T* p[kMaxOrder];
+};
+
+struct SpecPtrs {
+  const float2* p[kMaxOrder];   // spectrum blocks of filters 1..N
+};
+
+// Entry n of a kernel-parameter pointer array without a runtime-indexed copy
+// to local memory (every candidate is read straight from the parameter bank).
+template <typename A>
+__device__ __forceinline__ auto pick(const A& arr, int n) {
+  auto r = arr.p[0];
+#pragma unroll
+  for (int i = 1; i < kMaxOrder; ++i)
+    if (n == i) r = arr.p[i];
+  return r;
+}
+
+struct FusedLaunch {
+  const void* v;
+  const void* x[kMaxOrder];
+  SpecPtrs hh;
+  void* y;
+  const float2* tables;
+  int B, D, L, N;
+  bool bf16;
+};
+
+struct FourStepLaunch {
+  const void* v;
+  const void* x[kMaxOrder];
+  SpecPtrs hh;
+  void* y;
+  const float2* tables;
+  float2* scratch;
+  int B, D, L, N;
+  bool bf16;
+  long long ch0;     // first channel (c-major order) of this wave
+  int wave;          // channels in this wave
+};
+
+// Grid for a persistent kernel: SM count x resident CTAs per SM.
+cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int* grid);
+
+cudaError_t launch_fill_tables(float2* tables, const Layout& y, cudaStream_t s);
+cudaError_t launch_fused_forward(const FusedLaunch& p, int logMV, cudaStream_t s);
+cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* tables, int D, int L, int logMV,
+                                  cudaStream_t s);
+cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
+cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
+                                     const Layout& y, cudaStream_t s);
+cudaError_t launch_filter_generate(const float* W1, const float* b1, const float* W2, const float* b2,
+                                   const float* W3, const float* b3, int n_bands, int width, int N, int D,
+                                   int L, float alpha_lo, float alpha_hi, float* h, cudaStream_t s);
+
+}  // namespace hyena

@@ -1,0 +1,73 @@
+// layout.h -- how a problem of length L is split, and where the library keeps
+// its filter spectrum and FFT tables. Shared by host dispatch and kernels.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hyena {
+
+// Lengths up to this run the fused per-channel kernel (whole channel in shared
+// memory); longer ones run the four-step decomposition through a workspace.
+constexpr int kFusedMaxL = 8192;
+constexpr int kMinM = 128;          // smallest internal transform (zero-extended below)
+constexpr int kMaxL = 1 << 20;
+constexpr int kFourStepMaxMV = 4096;
+constexpr int kFourStepMinM1 = 16;
+
+struct Layout {
+  int L;        // caller's length
+  int M;        // packed complex points per channel (real length of the causal problem)
+  int M1;       // four-step column length (1 for the fused path)
+  int MV;       // row length, M = M1 * MV
+  int logMV;
+  int mb;       // M1 / 16 for the four-step path (radix of the second column pass)
+  bool fourstep;
+  // table region (float2 offsets from its start)
+  int tw_v;     // MV-point plan twiddles (MV entries)
+  int w_v;      // w_{2 MV}^k, k < MV
+  int tw_1;     // M1-point column plan twiddles (M1 entries, four-step only)
+  int table_len;
+};
+
+inline int ilog2_exact(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return ((1 << l) == v) ? l : -1;
+}
+
+// Returns false when L is not supported (not a power of two in [16, 2^20]).
+inline bool make_layout(int L, Layout* out) {
+  if (L < 16 || L > kMaxL) return false;
+  if (ilog2_exact(L) < 0) return false;
+  Layout y{};
+  y.L = L;
+  if (L <= kFusedMaxL) {
+    y.M = L < kMinM ? kMinM : L;
+    y.M1 = 1;
+    y.MV = y.M;
+    y.fourstep = false;
+    y.mb = 0;
+  } else {
+    y.M = L;
+    y.M1 = L / kFourStepMaxMV;
+    if (y.M1 < kFourStepMinM1) y.M1 = kFourStepMinM1;
+    y.MV = L / y.M1;
+    y.fourstep = true;
+    y.mb = y.M1 / 16;
+  }
+  y.logMV = ilog2_exact(y.MV);
+  y.tw_v = 0;
+  y.w_v = y.MV;
+  y.tw_1 = 2 * y.MV;
+  y.table_len = 2 * y.MV + (y.fourstep ? y.M1 : 0);
+  y.table_len = (y.table_len + 1) & ~1;   // keep the block a multiple of 16 bytes
+  *out = y;
+  return true;
+}
+
+// One filter's spectrum block: [D][M] float2 spectrum (library order) followed
+// by the table region.
+inline size_t spectrum_block_floats2(const Layout& y, int D) { return (size_t)D * y.M + y.table_len; }
+
+}  // namespace hyena

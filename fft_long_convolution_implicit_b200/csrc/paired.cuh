@@ -1,0 +1,149 @@
+// paired.cuh -- the pass where spectrum bins k and M-k meet.
+//
+// The last forward Stockham pass (radix 8, span MV/8) leaves butterfly j
+// holding bins j + r*MV/8. Butterfly j of one row and butterfly j' of the
+// mirror row hold mirror bins, so a thread that owns both can unpack the real
+// transform, multiply by the filter spectrum and repack without touching
+// shared memory; the first inverse (transposed) pass then runs on the same
+// registers. Mirror pairs are (a[r], b[7-r]) for every layout except the
+// head thread of row 0, whose butterflies 0 and MV/16 are each self-mirrored.
+#pragma once
+
+#include "fft_engine.cuh"
+
+namespace hyena {
+
+enum PairMode { kPairConv = 0, kPairSpectrum = 1 };
+
+// W for bin kA of row A: w_{2M}^{k1 + M1 k2} = rho * w_{2 MV}^{k2}.
+__device__ __forceinline__ float2 pair_w(const float2* __restrict__ Wv, int k2, float2 rho, bool has_rho) {
+  float2 w = __ldg(&Wv[k2]);
+  return has_rho ? cmul(rho, w) : w;
+}
+
+// MODE kPairConv: HA/HB are the spectrum rows of row A and row B (read);
+//   data is transformed in place in shared memory.
+// MODE kPairSpectrum: the unpacked spectrum 2 Z[k] * scale is written to HA/HB
+//   (library order, packed DC/Nyquist in bin 0 of row 0); shared memory is not
+//   written back.
+template <int LOGMV, int MODE>
+__device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA, int jB, bool head,
+                                            const float2* __restrict__ tw, const float2* __restrict__ Wv,
+                                            float2 rho, bool has_rho, float2* HA, float2* HB, float scale) {
+  constexpr int MV = 1 << LOGMV, Q8 = MV / 8, Q16 = MV / 16, NS = Q8;
+  float2 a[8], b[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    a[r] = baseA[pidx(jA + r * Q8)];
+    b[r] = baseB[pidx(jB + r * Q8)];
+  }
+  // filter spectrum for the product (loaded early: independent of the FFT)
+  float2 ha[8], hb[8];
+  if (MODE == kPairConv) {
+    if (!head) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        ha[r] = __ldg(&HA[jA + r * Q8]);
+        hb[r] = __ldg(&HB[jB + (7 - r) * Q8]);
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        ha[r] = __ldg(&HA[r * Q8]);
+        hb[r] = __ldg(&HA[Q16 + r * Q8]);
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 1; r < 8; ++r) {
+    a[r] = cmul(a[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jA]));
+    b[r] = cmul(b[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jB]));
+  }
+  dft8<false, 0>(a);
+  dft8<false, 0>(b);
+
+  if (!head) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int kA = jA + r * Q8;
+      const float2 W = pair_w(Wv, kA, rho, has_rho);
+      if (MODE == kPairConv) {
+        spectral_pair(a[r], b[7 - r], ha[r], hb[r], W);
+      } else {
+        float2 za, zb;
+        unpack_pair(a[r], b[7 - r], W, za, zb);
+        HA[kA] = make_float2(za.x * scale, za.y * scale);
+        HB[jB + (7 - r) * Q8] = make_float2(zb.x * scale, zb.y * scale);
+      }
+    }
+  } else {
+    // butterfly 0 of row 0: bins r*Q8. Bin 0 pairs with bin M (packed Nyquist),
+    // bin M/2 with itself, and r with 8-r otherwise.
+    {
+      const float2 one = make_float2(1.f, 0.f);
+      if (MODE == kPairConv) {
+        float2 c0 = a[0], c0b = a[0];
+        spectral_pair(c0, c0b, make_float2(ha[0].x, 0.f), make_float2(ha[0].y, 0.f), one);
+        a[0] = c0;
+      } else {
+        float2 za, zb;
+        unpack_pair(a[0], a[0], one, za, zb);
+        HA[0] = make_float2(za.x * scale, zb.x * scale);
+      }
+    }
+#pragma unroll
+    for (int r = 1; r < 4; ++r) {
+      const float2 W = __ldg(&Wv[r * Q8]);
+      if (MODE == kPairConv) {
+        spectral_pair(a[r], a[8 - r], ha[r], ha[8 - r], W);
+      } else {
+        float2 za, zb;
+        unpack_pair(a[r], a[8 - r], W, za, zb);
+        HA[r * Q8] = make_float2(za.x * scale, za.y * scale);
+        HA[(8 - r) * Q8] = make_float2(zb.x * scale, zb.y * scale);
+      }
+    }
+    {
+      const float2 W = __ldg(&Wv[4 * Q8]);
+      if (MODE == kPairConv) {
+        float2 c4 = a[4], c4b = a[4];
+        spectral_pair(c4, c4b, ha[4], ha[4], W);
+        a[4] = c4;
+      } else {
+        float2 za, zb;
+        unpack_pair(a[4], a[4], W, za, zb);
+        HA[4 * Q8] = make_float2(za.x * scale, za.y * scale);
+      }
+    }
+    // butterfly MV/16: bins Q16 + r*Q8, pairs r <-> 7-r
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float2 W = __ldg(&Wv[Q16 + r * Q8]);
+      if (MODE == kPairConv) {
+        spectral_pair(b[r], b[7 - r], hb[r], hb[7 - r], W);
+      } else {
+        float2 za, zb;
+        unpack_pair(b[r], b[7 - r], W, za, zb);
+        HA[Q16 + r * Q8] = make_float2(za.x * scale, za.y * scale);
+        HA[Q16 + (7 - r) * Q8] = make_float2(zb.x * scale, zb.y * scale);
+      }
+    }
+  }
+
+  if (MODE == kPairConv) {
+    dft8<true, 0>(a);
+    dft8<true, 0>(b);
+#pragma unroll
+    for (int r = 1; r < 8; ++r) {
+      a[r] = cmulc(a[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jA]));
+      b[r] = cmulc(b[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jB]));
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      baseA[pidx(jA + r * Q8)] = a[r];
+      baseB[pidx(jB + r * Q8)] = b[r];
+    }
+  }
+}
+
+}  // namespace hyena

@@ -1,0 +1,148 @@
+/*
+ * hyena.h -- C ABI of the B200 (sm_100a) Hyena order-N forward library.
+ *
+ * The operator (order-N recurrence; "Hyena Hierarchy - Towards Larger
+ * Convolutional Language Models" digest, section 방법 (Method) / 프레임워크
+ * 개요, and the explainer "Hyena Hierarchy: Towards Larger Convolutional
+ * Language Models", section Hyena 演算子の形):
+ *
+ *     z_1 = v,   z_{n+1} = x_n (.) (h_n * z_n),   y = z_{N+1},   n = 1..N
+ *
+ * where (.) is the elementwise product and * the causal long convolution
+ * (h * z)_t = sum_{s=0..t} h_{t-s} z_s ("02. 3つの Hyena 演算子", section 4,
+ * the FIR sum), evaluated by FFT on a 2L zero-padded grid (glossary
+ * "Hyena（ハイエナ）", section 計算効率; HyenaND summary, 境界の処理).
+ * The filters are implicit (glossary "Hyena（ハイエナ）", section
+ * 暗黙的畳み込みフィルタ: h(t) = Window(t) FFN(t/L, sin, cos)).
+ *
+ * Conventions for every call:
+ *  - Every pointer named "device" is CUDA device memory of the current
+ *    device, 16-byte aligned; the caller owns it. The library never
+ *    allocates device memory and keeps no state between calls.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream). Inputs must stay valid until the work on
+ *    the stream has finished.
+ *  - Arguments are checked on the host before anything is launched; a
+ *    rejected call launches nothing. HYENA_ERR_CUDA reports a launch error
+ *    (see hyena_last_cuda_error()).
+ *  - Activations v, x_n, y are row-major [B][D][L] (time fastest) in the
+ *    storage type `dtype`; the arithmetic is float32 throughout and bf16
+ *    results are rounded to nearest even.
+ *  - L must be a power of two with 16 <= L <= 2^20 (HYENA_ERR_UNSUPPORTED
+ *    otherwise); 1 <= N <= 8; B, D >= 1.
+ *  - All entry points are thread-safe.
+ */
+#ifndef HYENA_B200_H
+#define HYENA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HYENA_ABI_VERSION 1
+
+typedef enum {
+  HYENA_OK = 0,
+  HYENA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad count or dtype */
+  HYENA_ERR_UNSUPPORTED = 2,   /* L not a power of two in [16, 2^20] */
+  HYENA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  HYENA_ERR_CUDA = 4           /* a CUDA launch or attribute call failed */
+} hyena_status;
+
+typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype;
+
+typedef void *hyena_stream; /* cudaStream_t */
+
+/*
+ * Weights of the implicit-filter FFN, device float32, row-major [out][in]:
+ *   W1 [width][1 + 2 n_bands], b1 [width]
+ *   W2 [width][width],          b2 [width]
+ *   W3 [N*D][width],            b3 [N*D]
+ * n_bands in [1, 32], width in [1, 128].
+ */
+typedef struct {
+  const float *W1, *b1, *W2, *b2, *W3, *b3;
+  int n_bands;
+  int width;
+} hyena_filter_params;
+
+/*
+ * hyena_filter_generate -- implicit filters h_1..h_N.
+ * Glossary "Hyena（ハイエナ）", section 暗黙的畳み込みフィルタ; the workload
+ * recipe fixes the details:
+ *   e(t) = [t/L, sin(2 pi k t/L) for k = 1..K, cos(2 pi k t/L) for k = 1..K]
+ *   s1 = sin(W1 e + b1), s2 = sin(W2 s1 + b2), o = W3 s2 + b3
+ *   h[n][c][t] = o[n*D + c] * exp(-alpha_c t / L),
+ *   alpha_c = alpha_lo + (alpha_hi - alpha_lo) c / (D - 1)   (alpha_lo if D = 1)
+ * Output h: device float32 [N][D][L]. Returns HYENA_ERR_UNSUPPORTED for an
+ * unsupported L.
+ */
+hyena_status hyena_filter_generate(const hyena_filter_params *p, int N, int D, int L, float alpha_lo,
+                                   float alpha_hi, float *h, hyena_stream stream);
+
+/*
+ * Bytes of one filter's spectrum block for D channels and length L: the
+ * spectrum in library order plus the FFT tables the forward reads. 0 when L
+ * is unsupported or D < 1.
+ */
+size_t hyena_filter_spectrum_bytes(int D, int L);
+
+/*
+ * hyena_filter_rfft -- cache the spectrum of ONE filter (D channels):
+ *   H_c[k] = sum_{t<L} h_c[t] exp(-2 pi i k t / 2L) / (4 M),  k = 0..M,
+ * with M = max(L, 128) (rfft of the filter zero-padded to the 2L grid; the
+ * 1/(4M) folds the inverse transform's scale). Input h: device float32
+ * [D][L] (for example h + n*D*L from hyena_filter_generate). Output hhat:
+ * device block of hyena_filter_spectrum_bytes(D, L) bytes, library order
+ * (see hyena_spectrum_layout). Call once per filter n; reuse for every
+ * forward with the same weights.
+ */
+hyena_status hyena_filter_rfft(const float *h, int D, int L, void *hhat, hyena_stream stream);
+
+/*
+ * Describe the library order of a spectrum block (for inspection and tests):
+ * *M = points per channel, bin k < M of channel c sits at float2 index
+ * c*M + (k mod M1)*MV + (k / M1); bin 0 holds (Re H[0], Re H[M]). Returns
+ * HYENA_ERR_UNSUPPORTED for an unsupported L.
+ */
+hyena_status hyena_spectrum_layout(int L, int *M, int *M1, int *MV);
+
+/*
+ * Workspace bytes hyena_forward wants for this shape: 0 for L <= 8192 (the
+ * fused kernel keeps everything on chip); for longer L, 8*L bytes per
+ * channel for a wave of channels sized to stay resident in L2. Any workspace
+ * of at least 8*L bytes works (smaller waves); 0 when the shape is invalid.
+ */
+size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dtype);
+
+/*
+ * hyena_forward -- y = z_{N+1} of the order-N recurrence.
+ *   v:    device [B][D][L] dtype
+ *   x:    host array of N device pointers, x[n] = gate x_{n+1}, [B][D][L] dtype
+ *   hhat: host array of N device pointers to spectrum blocks from
+ *         hyena_filter_rfft (D channels, the same L)
+ *   y:    device [B][D][L] dtype; may alias v or any x[n] (each element is
+ *         read before the same thread block writes it)
+ *   workspace: device scratch of workspace_bytes (>= 8*L when L > 8192;
+ *         ignored otherwise, may be NULL)
+ */
+hyena_status hyena_forward(const void *v, const void *const *x, const void *const *hhat, int B, int D, int L,
+                           int N, hyena_dtype dtype, void *y, void *workspace, size_t workspace_bytes,
+                           hyena_stream stream);
+
+/* Static description of a status code. */
+const char *hyena_status_string(hyena_status s);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char *hyena_last_cuda_error(void);
+
+/* HYENA_ABI_VERSION of the loaded library. */
+int hyena_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HYENA_B200_H */

@@ -1,0 +1,95 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every
+function include/hyena.h declares, and rejects bad arguments on the host
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fft_long_convolution_implicit_b200 as hy
+from fft_long_convolution_implicit_b200 import build as hybuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hybuild.build()
+    return hy.load()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(hyena_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_binding_exports():
+    assert set(declared_functions()) == set(hy.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_host_queries(lib):
+    assert hy.abi_version() == 1
+    assert lib.hyena_status_string(0) == b"ok"
+    # spectrum block: D*M complex64 + tables
+    M, M1, MV = hy.spectrum_layout(2048)
+    assert (M, M1, MV) == (2048, 1, 2048)
+    assert hy.filter_spectrum_bytes(768, 2048) >= 768 * 2048 * 8
+    assert hy.spectrum_layout(16)[0] == 128                  # small L is zero-extended to 128 points
+    M, M1, MV = hy.spectrum_layout(1 << 20)
+    assert M == 1 << 20 and M1 * MV == M and MV <= 4096
+    M, M1, MV = hy.spectrum_layout(131072)
+    assert (M1, MV) == (32, 4096)
+    assert hy.forward_workspace_bytes(4, 768, 2048, 2, True) == 0
+    ws = hy.forward_workspace_bytes(1, 256, 131072, 2, True)
+    assert ws % (131072 * 8) == 0 and ws >= 131072 * 8
+    assert hy.forward_workspace_bytes(1, 1, 1000, 2, True) == 0       # unsupported L
+    assert hy.filter_spectrum_bytes(4, 3000) == 0
+
+
+@pytest.mark.parametrize("L", [0, 8, 1000, 3 << 10, 1 << 21])
+def test_unsupported_lengths_rejected_before_launch(lib, L):
+    p = ctypes.c_void_p(16)      # never dereferenced: the call must fail on the host
+    xs = (ctypes.c_void_p * 2)(16, 16)
+    st = lib.hyena_forward(p, xs, xs, 1, 1, L, 2, hy.HYENA_BF16, p, None, 0, None)
+    assert st == hy.HYENA_ERR_UNSUPPORTED
+    assert lib.hyena_filter_rfft(p, 1, L, p, None) == hy.HYENA_ERR_UNSUPPORTED
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    p = ctypes.c_void_p(16)
+    xs = (ctypes.c_void_p * 2)(16, 16)
+    f = lib.hyena_forward
+    assert f(None, xs, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, None, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1024, 0, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1024, 9, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 0, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1024, 2, 7, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    mis = ctypes.c_void_p(24)    # 8-byte aligned only
+    assert f(mis, xs, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    # long L needs a workspace of at least 8 L bytes
+    assert f(p, xs, xs, 1, 1, 1 << 15, 2, 0, p, None, 0, None) == hy.HYENA_ERR_WORKSPACE
+    assert f(p, xs, xs, 1, 1, 1 << 15, 2, 0, p, p, 8 * (1 << 15) - 16, None) == hy.HYENA_ERR_WORKSPACE
+    fp = hy.FilterParams(16, 16, 16, 16, 16, 16, 8, 64)
+    g = lib.hyena_filter_generate
+    assert g(None, 2, 4, 1024, 0.5, 20.0, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert g(ctypes.byref(fp), 2, 4, 1000, 0.5, 20.0, p, None) == hy.HYENA_ERR_UNSUPPORTED
+    bad = hy.FilterParams(16, 16, 16, 16, 16, 16, 8, 512)
+    assert g(ctypes.byref(bad), 2, 4, 1024, 0.5, 20.0, p, None) == hy.HYENA_ERR_INVALID_ARG
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.hyena_status_string(s)
+    assert lib.hyena_last_cuda_error() == b""

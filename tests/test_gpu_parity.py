@@ -1,0 +1,166 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Tolerance: per (b, c) row relative L2 error <= 2e-5 for float32 I/O and
+<= 8e-3 for bfloat16 I/O (float32 arithmetic inside, bf16 output rounding).
+Small shapes are compared on every row; the five workloads at full size are
+run in the same launch configuration as the benchmark and compared on a
+seeded sample of rows (always including the first and the last).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from hyena_cases import TOL, gpu_run, oracle_rows, rel_l2_rows, upload, weights_to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def hy():
+    from fft_long_convolution_implicit_b200 import build
+    build.build()
+    import fft_long_convolution_implicit_b200 as m
+    m.load()
+    return m
+
+
+# ------------------------------------------------------------ filter gen ---
+
+@pytest.mark.parametrize("cfg_i", [0, 1, 3])
+def test_filter_generate_matches_oracle(hy, cfg_i):
+    w = synth.workload(cfg_i)
+    wt = synth.filter_weights(w)
+    h = hy.filter_generate(weights_to_cuda(wt), w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
+    hg = h.cpu().numpy().reshape(w.N * w.D, w.L)
+    cs = range(w.D) if w.D <= 16 else [0, 1, w.D // 2, w.D - 1]
+    rows = [(n, c) for n in range(w.N) for c in cs]
+    ref = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi, rows=rows)
+    got = np.stack([hg[n * w.D + c] for n, c in rows])
+    err = rel_l2_rows(got, ref)
+    assert err.max() < 1e-6, err.max()
+
+
+# -------------------------------------------------------------- spectrum ---
+
+@pytest.mark.parametrize("L", [16, 128, 1024, 2048, 8192, 16384, 65536, 131072])
+def test_spectrum_matches_oracle(hy, L):
+    import torch
+    rng = np.random.default_rng(L)
+    D = 3
+    h = (rng.standard_normal((D, L)) * np.exp(-np.arange(L) / (0.2 * L))).astype(np.float32)
+    hh = hy.filter_rfft(torch.from_numpy(h).cuda())
+    nat = hy.spectrum_natural(hh, D, L).cpu().numpy()
+    M = max(L, 128)
+    for c in range(D):
+        hp = np.zeros(M); hp[:L] = h[c]
+        ref = oracle.filter_spectrum(hp) / (4 * M)
+        err = np.linalg.norm(nat[c] - ref) / np.linalg.norm(ref)
+        assert err < 2e-6, (c, err)
+
+
+# ------------------------------------------------------- forward parity ---
+
+@pytest.mark.parametrize("cfg_i,nsample", [(0, None), (1, 24), (2, 12), (3, 6), (4, 3)])
+def test_forward_workload(hy, cfg_i, nsample):
+    w = synth.workload(cfg_i)
+    y, _, (v, xs, wt) = gpu_run(w)
+    assert np.isfinite(y).all()
+    rows = list(range(w.channels)) if nsample is None else synth.sample_rows(w, nsample)
+    ref = oracle_rows(w, rows, v, xs, wt)
+    err = rel_l2_rows(y[rows], ref)
+    assert err.max() <= TOL[w.dtype], (err.max(), rows[int(np.argmax(err))])
+
+
+SWEEP = [
+    # N, dtype, B, D, L
+    (1, "f32", 1, 1, 16),
+    (2, "f32", 3, 5, 32),
+    (3, "f32", 1, 2, 64),
+    (4, "f32", 2, 3, 128),
+    (2, "f32", 1, 4, 256),
+    (2, "bf16", 3, 5, 512),
+    (3, "f32", 2, 2, 1024),
+    (1, "f32", 2, 2, 4096),
+    (2, "f32", 1, 3, 8192),
+    (2, "f32", 1, 2, 16384),
+    (3, "bf16", 1, 3, 32768),
+    (2, "f32", 2, 1, 65536),
+    (1, "f32", 1, 2, 262144),
+    (2, "bf16", 1, 2, 524288),
+]
+
+
+@pytest.mark.parametrize("N,dtype,B,D,L", SWEEP)
+def test_forward_shapes(hy, N, dtype, B, D, L):
+    w = synth.custom(N, dtype, B, D, L, seed=11 + L + N)
+    y, _, (v, xs, wt) = gpu_run(w)
+    rows = list(range(w.channels))
+    ref = oracle_rows(w, rows, v, xs, wt)
+    err = rel_l2_rows(y, ref)
+    assert err.max() <= TOL[dtype], err.max()
+
+
+@pytest.mark.parametrize("L", [2048, 32768])
+def test_forward_in_place_and_waves(hy, L):
+    import torch
+    w = synth.custom(2, "f32", 2, 3, L, seed=5)
+    y_ref, _, (v, xs, wt) = gpu_run(w)
+    tw = weights_to_cuda(wt)
+    h = hy.filter_generate(tw, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
+    hh = [hy.filter_rfft(h[n]) for n in range(w.N)]
+    # y aliasing v
+    tv = upload(v, w)
+    txs = [upload(x, w) for x in xs]
+    hy.forward(tv, txs, hh, y=tv)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(tv.cpu().numpy().reshape(w.channels, L), y_ref)
+    # y aliasing the last gate
+    tv = upload(v, w)
+    hy.forward(tv, txs, hh, y=txs[-1])
+    np.testing.assert_array_equal(txs[-1].cpu().numpy().reshape(w.channels, L), y_ref)
+    if L > 8192:
+        # a one-channel workspace: every channel runs in its own wave
+        tv = upload(v, w)
+        txs = [upload(x, w) for x in xs]
+        ws = torch.empty(8 * L, dtype=torch.uint8, device="cuda")
+        y1 = hy.forward(tv, txs, hh, workspace=ws)
+        np.testing.assert_array_equal(y1.cpu().numpy().reshape(w.channels, L), y_ref)
+
+
+@pytest.mark.parametrize("cfg_i", [1, 2, 3, 4])
+def test_full_size_delta_filter_identity(hy, cfg_i):
+    """With every h_n = delta the recurrence is y = v * x_1 * ... * x_N: checks
+    the whole transform round trip on every row at full size."""
+    import torch
+    w = synth.workload(cfg_i)
+    g = torch.Generator(device="cuda").manual_seed(cfg_i)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    v = torch.randn(w.B, w.D, w.L, device="cuda", generator=g).to(dt)
+    xs = [torch.randn(w.B, w.D, w.L, device="cuda", generator=g).to(dt) for _ in range(w.N)]
+    h = torch.zeros(w.D, w.L, device="cuda")
+    h[:, 0] = 1.0
+    hh = hy.filter_rfft(h)
+    y = hy.forward(v, xs, [hh] * w.N).double()
+    ref = v.double()
+    for x in xs:
+        ref = ref * x.double()
+    num = torch.linalg.vector_norm(y - ref, dim=-1)
+    den = torch.linalg.vector_norm(ref, dim=-1)
+    assert (num / den).max().item() <= TOL[w.dtype]
+
+
+def test_forward_is_deterministic_and_scales_exactly(hy):
+    import torch
+    w = synth.workload(2)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    tv = torch.randn(w.B, w.D, w.L, device="cuda", generator=g).bfloat16()
+    txs = [torch.randn(w.B, w.D, w.L, device="cuda", generator=g).bfloat16() for _ in range(w.N)]
+    wt = synth.filter_weights(w)
+    h = hy.filter_generate(weights_to_cuda(wt), w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
+    hh = [hy.filter_rfft(h[n]) for n in range(w.N)]
+    y1 = hy.forward(tv, txs, hh)
+    y2 = hy.forward(tv, txs, hh)
+    y4 = hy.forward(tv * 4, txs, hh)
+    assert torch.equal(y1, y2)
+    assert torch.equal(y4, y1 * 4)
