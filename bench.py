@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Benchmark of the Hyena order-N forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
+
+A step is one hyena_forward over one batch of the workload (default: the
+order-2, bf16, B=4, D=768, L=2048 workload), with the filter spectra already
+cached (they depend only on the weights). Inputs are resident in HBM when the
+timed region starts and are rotated over enough buffer sets that the step's
+working set is not in L2. The metric is B*D*L processed per second (x1e9)
+and the fraction of the HBM roofline; one JSON line is printed by rank 0.
+
+--gpus N > 1 runs under torchrun: every rank processes its own batch
+(weak scaling, no collective on the data path); time is the max over ranks.
+--impl reference times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "Hyena order-N fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
+UNIT = "1e9 B*D*L/s"
+KERNEL_SOURCES = os.path.join(ROOT, "fft_long_convolution_implicit_b200", "csrc")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for fn in sorted(os.listdir(KERNEL_SOURCES)):
+        with open(os.path.join(KERNEL_SOURCES, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_traffic(workload_name: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    capture, or None when absent or taken on different kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        e = t.get(workload_name)
+        if e and e.get("source_sha") == kernel_source_sha():
+            return int(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------ clocks -----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------- oracle arm --
+
+def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0):
+    """Time the float64 oracle (as it stands) on a bounded sample of rows of
+    the workload; filters are computed beforehand and not timed."""
+    import oracle
+    threads = host_cores()
+    wt = synth.filter_weights(w)
+    # calibrate: one row, then size the sample for ~target core-seconds
+    probe_rows = [0]
+    v, xs = synth.inputs(w, probe_rows)
+    cs = [0]
+    hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
+                                   rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
+    hs = [hrows[n:n + 1] for n in range(w.N)]
+    t0 = time.perf_counter()
+    oracle.hyena_forward(v, xs, hs, threads=1)
+    per_row = max(time.perf_counter() - t0, 1e-4)
+    nrows = int(min(w.channels, max(threads, target_core_seconds / per_row)))
+    rows = list(range(nrows))
+    v, xs = synth.inputs(w, rows)
+    cs = sorted({r % w.D for r in rows})
+    hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
+                                   rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
+    hs = [hrows[n * len(cs):(n + 1) * len(cs)] for n in range(w.N)]
+    fr = [cs.index(r % w.D) for r in rows]
+    t0 = time.perf_counter()
+    oracle.hyena_forward(v, xs, hs, filter_row=fr, threads=threads)
+    dt = time.perf_counter() - t0
+    value = nrows * w.L / dt / 1e9
+    sample = (f"{nrows} of {w.channels} (b,c) rows of {w.name}, all N={w.N} stages, "
+              f"{'direct O(L^2)' if w.L <= 8192 else 'radix-2 FFT'} causal conv, filters precomputed")
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+            "seconds": dt}
+
+
+# ---------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1, help="workload index (default 1: B=4 D=768 L=2048 N=2 bf16)")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    w = synth.workload(args.config)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = oracle_sample(w)
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.channels * w.L / (cb["value"] * 1e9) * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N,
+                                                 "io": w.dtype},
+                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    import fft_long_convolution_implicit_b200 as hy
+    from fft_long_convolution_implicit_b200 import build as hybuild
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        hybuild.build()
+    if world > 1:
+        dist.barrier()
+    hy.load()
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+
+    # inputs of this rank (seeded per rank), weights and cached spectra
+    wr = synth.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
+    v_np, xs_np = synth.inputs(wr)
+    wt = synth.filter_weights(wr)
+    tw = {k: torch.from_numpy(np.ascontiguousarray(a)).to(dev) for k, a in wt.items()}
+    h = hy.filter_generate(tw, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
+    base_v = torch.from_numpy(v_np).view(w.B, w.D, w.L).to(dev).to(dt)
+    base_x = [torch.from_numpy(x).view(w.B, w.D, w.L).to(dev).to(dt) for x in xs_np]
+    base_h = [hy.filter_rfft(h[n]) for n in range(w.N)]
+    del h
+    set_bytes = (w.N + 2) * w.channels * w.L * w.elem_bytes + sum(t.numel() for t in base_h)
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    sets = []
+    for s in range(nsets):
+        if s == 0:
+            v_s, x_s, h_s = base_v, base_x, base_h
+        else:
+            v_s, x_s, h_s = base_v.clone(), [x.clone() for x in base_x], [t.clone() for t in base_h]
+        sets.append(hy.PreparedForward(v_s, x_s, h_s, stream=stream))
+    torch.cuda.synchronize()
+    launches_per_step = 1 if w.L <= 8192 else None
+    if launches_per_step is None:
+        M, M1, MV = hy.spectrum_layout(w.L)
+        ws = hy.forward_workspace_bytes(w.B, w.D, w.L, w.N, dt == torch.bfloat16)
+        wave = ws // (8 * w.L)
+        waves = math.ceil(w.channels / wave)
+        launches_per_step = waves * (2 * w.N + 1)
+
+    # warm-up
+    for i in range(args.warmup):
+        sets[i % nsets]()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.2)
+    K = args.steps
+    ev_pre = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_post = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        ev_pre[i].record(stream)
+        sets[i % nsets]()
+        ev_post[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev_pre, ev_post)]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    units = K * w.channels * w.L * world
+    value = units / (elapsed_ms * 1e-3) / 1e9
+    kernel_ms = statistics.mean(step_ms)
+    peak, peak_kind = hbm_peak()
+    alg_bytes = w.roofline_bytes()
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs in, result out
+    pin_v = base_v.cpu().pin_memory()
+    pin_x = [x.cpu().pin_memory() for x in base_x]
+    pin_y = torch.empty_like(pin_v).pin_memory()
+    dv = torch.empty_like(base_v)
+    dxs = [torch.empty_like(x) for x in base_x]
+    e2e_fwd = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream)
+    h2d = (w.N + 1) * w.channels * w.L * w.elem_bytes
+    d2h = w.channels * w.L * w.elem_bytes
+
+    def e2e_step():
+        dv.copy_(pin_v, non_blocking=True)
+        for d, p in zip(dxs, pin_x):
+            d.copy_(p, non_blocking=True)
+        y = e2e_fwd()
+        pin_y.copy_(y, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = args.e2e_steps * w.channels * w.L * world / (e2e_ms * 1e-3) / 1e9
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype,
+                       "global_batch": w.B * world, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
+                             f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
+                         "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
+                         "kernel": "fused_forward_kernel" if w.L <= 8192 else "whole step (four-step kernels)",
+                         "kernel_ms": round(kernel_ms, 5)},
+            "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
+            "gpu_launches": K * launches_per_step,
+            "clocks": clocks,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            cb = oracle_sample(w)
+            line["cpu_baseline"] = {k: round(cb[k], 6) if k == "value" else cb[k]
+                                    for k in ("value", "unit", "cores", "kind", "sample")}
+        elif not args.no_cpu_baseline:
+            line["cpu_baseline"] = None
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
