@@ -25,7 +25,7 @@ HYENA_F32, HYENA_BF16 = 0, 1
 EXPORTS = (
     "hyena_filter_generate", "hyena_filter_spectrum_bytes", "hyena_filter_rfft", "hyena_spectrum_layout",
     "hyena_forward_workspace_bytes", "hyena_forward", "hyena_status_string", "hyena_last_cuda_error",
-    "hyena_abi_version",
+    "hyena_abi_version", "hyena_forward_static_workspace",
 )
 
 
@@ -70,6 +70,8 @@ def load() -> ctypes.CDLL:
     l.hyena_forward_workspace_bytes.restype = sz
     l.hyena_forward.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
     l.hyena_forward.restype = i
+    l.hyena_forward_static_workspace.argtypes = [P, P, P, i, i, i, i, i, P, P]
+    l.hyena_forward_static_workspace.restype = i
     l.hyena_status_string.argtypes = [i]
     l.hyena_status_string.restype = ctypes.c_char_p
     l.hyena_last_cuda_error.argtypes = []
@@ -187,6 +189,27 @@ def forward(v, xs, hhats, y=None, workspace=None, stream=None):
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().hyena_forward(_dev(v, "v"), xarr, harr, B, D, L, N, code, _dev(y, "y"), ws_ptr, ws_bytes,
                                 _stream(stream)), "hyena_forward")
+    return y
+
+
+def forward_static_workspace(v, xs, hhats, y=None, stream=None):
+    """hyena_forward_static_workspace: the long-sequence forward (8192 < L)
+    with the library's static device scratch instead of a caller workspace,
+    for callers that cannot allocate device memory. Calls whose GPU work
+    overlaps race on that scratch; the first call on a device must come
+    before any stream capture on it."""
+    torch = _torch()
+    B, D, L = v.shape
+    N = len(xs)
+    if len(hhats) != N:
+        raise ValueError("need one spectrum per gate")
+    code = _dtype_code(v)
+    if y is None:
+        y = torch.empty_like(v)
+    xarr = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+    harr = (ctypes.c_void_p * N)(*[_dev(hh, "hhat").value for hh in hhats])
+    _check(load().hyena_forward_static_workspace(_dev(v, "v"), xarr, harr, B, D, L, N, code, _dev(y, "y"),
+                                                 _stream(stream)), "hyena_forward_static_workspace")
     return y
 
 

@@ -42,6 +42,8 @@ std::unordered_map<GridKey, int, GridKeyHash> g_grid_cache;
 
 }  // namespace
 
+hyena_status hyena::report_cuda_error(cudaError_t e) { return cuda_fail(e); }
+
 cudaError_t hyena::persistent_grid(const void* kernel, int threads, size_t smem, int* grid) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "hyena.h"
 #include "layout.h"
 
 namespace hyena {
@@ -53,6 +54,10 @@ struct FourStepLaunch {
   long long ch0;     // first channel (c-major order) of this wave
   int wave;          // channels in this wave
 };
+
+// Records e as this thread's last CUDA error (hyena_last_cuda_error) and
+// returns HYENA_ERR_CUDA.
+hyena_status report_cuda_error(cudaError_t e);
 
 // Grid for a persistent kernel: SM count x resident CTAs per SM.
 cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int* grid);

@@ -132,6 +132,40 @@ hyena_status hyena_forward(const void *v, const void *const *x, const void *cons
                            int N, hyena_dtype dtype, void *y, void *workspace, size_t workspace_bytes,
                            hyena_stream stream);
 
+/*
+ * hyena_forward_static_workspace -- hyena_forward for callers that cannot
+ * allocate device memory (no counterpart on the pages: it is a deployment
+ * convenience, not part of the method).
+ *
+ * Some callers may not call cudaMalloc at run time: runtimes that own the
+ * whole device through their own pool allocator and forbid allocations
+ * behind its back, fixed-budget deployments, and latency-critical paths that
+ * cannot afford cudaMalloc's implicit device synchronisation. This entry point
+ * needs no workspace argument: the four-step scratch lives in a file-scope
+ * device array of HYENA_STATIC_WORKSPACE_BYTES inside the library, reserved
+ * on every GPU that loads the library and held until the process exits.
+ * It allocates nothing and calls no allocating routine.
+ *
+ *  - Only for 8192 < L <= 2^20 (the lengths whose forward needs scratch);
+ *    shorter L returns HYENA_ERR_UNSUPPORTED: use hyena_forward with a NULL
+ *    workspace there, which already allocates nothing.
+ *  - Channels are processed in waves of HYENA_STATIC_WORKSPACE_BYTES / (8 L);
+ *    a length whose single channel would not fit is rejected with
+ *    HYENA_ERR_WORKSPACE (never the case for supported L).
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - Every call on a device shares the one array and leaves its last
+ *    contents there (nothing needs clearing: every element is written before
+ *    it is read). Calls whose GPU work overlaps -- on different streams, or
+ *    from different threads -- race on the array: order them on one stream
+ *    or otherwise serialise them.
+ * Other arguments, layouts and errors are those of hyena_forward.
+ */
+#define HYENA_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+hyena_status hyena_forward_static_workspace(const void *v, const void *const *x, const void *const *hhat, int B,
+                                            int D, int L, int N, hyena_dtype dtype, void *y, hyena_stream stream);
+
 /* Static description of a status code. */
 const char *hyena_status_string(hyena_status s);
 
