@@ -44,9 +44,16 @@ FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2 ** 20
 
 
-def kernel_source_sha() -> str:
+# sources the dominant kernel of each path is compiled from
+KERNEL_FILES = {
+    "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
+    "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
+}
+
+
+def kernel_source_sha(path: str = "fused") -> str:
     h = hashlib.sha256()
-    for fn in sorted(os.listdir(KERNEL_SOURCES)):
+    for fn in KERNEL_FILES[path]:
         with open(os.path.join(KERNEL_SOURCES, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -67,7 +74,7 @@ def measured_traffic(workload_name: str):
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
         e = t.get(workload_name)
-        if e and e.get("source_sha") == kernel_source_sha():
+        if e and e.get("source_sha") == kernel_source_sha(e.get("path", "fused")):
             return int(e["dram_bytes_per_launch"])
     except Exception:
         pass
