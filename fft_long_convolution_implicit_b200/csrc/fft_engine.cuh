@@ -156,11 +156,37 @@ __device__ __forceinline__ void dftR(float2 (&a)[N]) {
   else static_assert(R == 2 || R == 4 || R == 8 || R == 16, "radix");
 }
 
+// ------------------------------------------------------------ async copy --
+// 16-byte global -> shared copies that complete asynchronously (cp.async,
+// L2 only); completion is awaited with the hardware group wait, no polling.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// Copy nbytes (multiple of 16, both addresses 16-byte aligned) with all
+// threads of the block; returns without waiting.
+__device__ __forceinline__ void block_copy_async(void* smem_dst, const void* gmem_src, int nbytes, int tid,
+                                                 int nthreads) {
+  char* d = reinterpret_cast<char*>(smem_dst);
+  const char* g = reinterpret_cast<const char*>(gmem_src);
+  for (int off = tid * 16; off < nbytes; off += nthreads * 16) cp_async16(d + off, g + off);
+}
+
 // ----------------------------------------------------------- smem padding --
 // one float2 of padding after every 16: removes the bank conflicts of the
 // stride-16 block writes of radix-16 passes
 __device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
 __host__ __device__ constexpr int padded_len(int m) { return m + m / 16; }
+// pidx(i + r*STEP) from p = pidx(i): a compile-time offset when STEP is a
+// multiple of 16 (adding whole 16-element groups moves the padding exactly).
+template <int STEP>
+__device__ __forceinline__ int pidx_step(int p, int i, int r) {
+  if constexpr (STEP % 16 == 0) return p + r * (STEP + STEP / 16);
+  else return pidx(i + r * STEP);
+}
 
 // ---------------------------------------------------------------- plans ----
 // Pass plan of an MV-point FFT (MV = 2^LOGMV, LOGMV >= 7), 16 points per
@@ -197,15 +223,17 @@ __device__ __forceinline__ void dft_blocks(float2 (&a)[16]) {
 template <int LOGMV, int I>
 __device__ __forceinline__ void mid_fwd(float2 (&a)[16], float2* base, const float2* __restrict__ tw, int tl) {
   using P = Plan<LOGMV>;
-  constexpr int MV = P::MV, TV = P::TV, R = P::radix(I), NS = P::span(I), NB = 16 / R;
+  constexpr int MV = P::MV, TV = P::TV, R = P::radix(I), NS = P::span(I), NB = 16 / R, S = MV / R;
+  const int ptl = pidx(tl);
 #pragma unroll
   for (int q = 0; q < NB; ++q) {
     const int j = tl + q * TV;
+    const int pj = pidx_step<TV>(ptl, tl, q);
 #pragma unroll
-    for (int r = 0; r < R; ++r) a[q * R + r] = base[pidx(j + r * (MV / R))];
-    const int jm = j & (NS - 1);
+    for (int r = 0; r < R; ++r) a[q * R + r] = base[pidx_step<S>(pj, j, r)];
+    const float2* __restrict__ t = tw + (NS - 1) + (j & (NS - 1));
 #pragma unroll
-    for (int r = 1; r < R; ++r) a[q * R + r] = cmul(a[q * R + r], __ldg(&tw[NS - 1 + (r - 1) * NS + jm]));
+    for (int r = 1; r < R; ++r) a[q * R + r] = cmul(a[q * R + r], __ldg(t + (r - 1) * NS));
   }
   dft_blocks<R, false>(a);
   __syncthreads();
@@ -213,8 +241,9 @@ __device__ __forceinline__ void mid_fwd(float2 (&a)[16], float2* base, const flo
   for (int q = 0; q < NB; ++q) {
     const int j = tl + q * TV;
     const int o = (j / NS) * NS * R + (j & (NS - 1));
+    const int po = pidx(o);
 #pragma unroll
-    for (int r = 0; r < R; ++r) base[pidx(o + r * NS)] = a[q * R + r];
+    for (int r = 0; r < R; ++r) base[pidx_step<NS>(po, o, r)] = a[q * R + r];
   }
   __syncthreads();
 }
@@ -224,29 +253,45 @@ __device__ __forceinline__ void mid_fwd(float2 (&a)[16], float2* base, const flo
 template <int LOGMV, int I>
 __device__ __forceinline__ void mid_inv(float2 (&a)[16], float2* base, const float2* __restrict__ tw, int tl) {
   using P = Plan<LOGMV>;
-  constexpr int MV = P::MV, TV = P::TV, R = P::radix(I), NS = P::span(I), NB = 16 / R;
+  constexpr int MV = P::MV, TV = P::TV, R = P::radix(I), NS = P::span(I), NB = 16 / R, S = MV / R;
 #pragma unroll
   for (int q = 0; q < NB; ++q) {
     const int j = tl + q * TV;
     const int o = (j / NS) * NS * R + (j & (NS - 1));
+    const int po = pidx(o);
 #pragma unroll
-    for (int r = 0; r < R; ++r) a[q * R + r] = base[pidx(o + r * NS)];
+    for (int r = 0; r < R; ++r) a[q * R + r] = base[pidx_step<NS>(po, o, r)];
   }
   dft_blocks<R, true>(a);
 #pragma unroll
   for (int q = 0; q < NB; ++q) {
-    const int jm = (tl + q * TV) & (NS - 1);
+    const float2* __restrict__ t = tw + (NS - 1) + ((tl + q * TV) & (NS - 1));
 #pragma unroll
-    for (int r = 1; r < R; ++r) a[q * R + r] = cmulc(a[q * R + r], __ldg(&tw[NS - 1 + (r - 1) * NS + jm]));
+    for (int r = 1; r < R; ++r) a[q * R + r] = cmulc(a[q * R + r], __ldg(t + (r - 1) * NS));
   }
   __syncthreads();
+  const int ptl = pidx(tl);
 #pragma unroll
   for (int q = 0; q < NB; ++q) {
     const int j = tl + q * TV;
+    const int pj = pidx_step<TV>(ptl, tl, q);
 #pragma unroll
-    for (int r = 0; r < R; ++r) base[pidx(j + r * (MV / R))] = a[q * R + r];
+    for (int r = 0; r < R; ++r) base[pidx_step<S>(pj, j, r)] = a[q * R + r];
   }
   __syncthreads();
+}
+
+// First forward pass output / last inverse pass input of thread tl: the 16
+// positions 16 tl + r, padded index 17 tl + r.
+__device__ __forceinline__ void store_block16(float2* base, int tl, const float2 (&a)[16]) {
+  float2* p = base + 17 * tl;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) p[r] = a[r];
+}
+__device__ __forceinline__ void load_block16(const float2* base, int tl, float2 (&a)[16]) {
+  const float2* p = base + 17 * tl;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) a[r] = p[r];
 }
 
 template <int LOGMV, int I = 0>
@@ -310,6 +355,7 @@ struct IO<float> {
     return __ldcs(reinterpret_cast<const float2*>(p));
   }
   static __device__ __forceinline__ void store2(float* p, float2 v) { __stcs(reinterpret_cast<float2*>(p), v); }
+  static __device__ __forceinline__ float2 load2_smem(const float* p) { return *reinterpret_cast<const float2*>(p); }
 };
 template <>
 struct IO<__nv_bfloat16> {
@@ -319,6 +365,10 @@ struct IO<__nv_bfloat16> {
   }
   static __device__ __forceinline__ float2 load2_stream(const __nv_bfloat16* p) {
     unsigned int u = __ldcs(reinterpret_cast<const unsigned int*>(p));
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+  static __device__ __forceinline__ float2 load2_smem(const __nv_bfloat16* p) {
+    unsigned int u = *reinterpret_cast<const unsigned int*>(p);
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
   }
   static __device__ __forceinline__ void store2(__nv_bfloat16* p, float2 v) {

@@ -170,8 +170,7 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
     }
   }
   dft16<false, false, false, 0>(a);
-#pragma unroll
-  for (int r = 0; r < 16; ++r) base[pidx(16 * tl + r)] = a[r];
+  store_block16(base, tl, a);
   __syncthreads();
   mid_fwd_all<LOGMV>(a, base, tw, tl);
 
@@ -207,8 +206,7 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
   if (MODE == kPairSpectrum) return;
   __syncthreads();
   mid_inv_all<LOGMV>(a, base, tw, tl);
-#pragma unroll
-  for (int r = 0; r < 16; ++r) a[r] = base[pidx(16 * tl + r)];
+  load_block16(base, tl, a);
   dft16<true, false, false, 0>(a);
   {
     float2 cur = tw0;

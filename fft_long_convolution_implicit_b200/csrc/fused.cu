@@ -13,13 +13,39 @@
 
 namespace hyena {
 
+// Resident CTAs per SM the register budget is sized for.
+#ifndef HYENA_FUSED_THREADS_PER_SM
+#define HYENA_FUSED_THREADS_PER_SM 512
+#endif
+template <int LOGMV>
+struct FusedOcc {
+  static constexpr int TV = Plan<LOGMV>::TV;
+  static constexpr int T = HYENA_FUSED_THREADS_PER_SM;
+  static constexpr int value = TV >= 512 ? 1 : (T / TV > 16 ? 16 : (T / TV < 1 ? 1 : T / TV));
+};
+
+// Shared memory: z (padded), staged filter spectrum row, staged gate row,
+// staged v row of the next channel.
 template <int LOGMV, typename T>
-__global__ void __launch_bounds__(Plan<LOGMV>::TV)
+struct FusedSmem {
+  static constexpr int MV = 1 << LOGMV;
+  static constexpr size_t z = sizeof(float2) * padded_len(MV);
+  static constexpr size_t h = sizeof(float2) * MV;
+  static constexpr size_t row = sizeof(T) * MV;      // L <= MV elements, 16-byte multiple
+  static constexpr size_t total = z + h + 2 * row;
+};
+
+template <int LOGMV, typename T>
+__global__ void __launch_bounds__(Plan<LOGMV>::TV, FusedOcc<LOGMV>::value)
 fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __restrict__ y,
                      const float2* __restrict__ tables, int B, int D, int L, int N) {
   using P = Plan<LOGMV>;
-  constexpr int MV = P::MV, Q8 = MV / 8, Q16 = MV / 16;
-  extern __shared__ float2 sm[];
+  using S = FusedSmem<LOGMV, T>;
+  constexpr int MV = P::MV, TV = P::TV, Q8 = MV / 8, Q16 = MV / 16;
+  extern __shared__ __align__(16) float2 sm[];
+  float2* hs = reinterpret_cast<float2*>(reinterpret_cast<char*>(sm) + S::z);
+  T* xs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h);
+  T* vs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h + S::row);
   const int tl = threadIdx.x;
   const float2* __restrict__ tw = tables;
   const float2* __restrict__ Wv = tables + MV;
@@ -28,39 +54,69 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
   const int jA = head ? 0 : tl;
   const int jB = head ? Q16 : Q8 - tl;
   const float2 one = make_float2(1.f, 0.f);
+  const int row_bytes = L * (int)sizeof(T);
+  const int h_bytes = MV * (int)sizeof(float2);
 
-  for (long long ch = blockIdx.x; ch < C; ch += gridDim.x) {
-    // channel order c-major so that CTAs sharing a filter run side by side
+  // channel order c-major so that CTAs sharing a filter run side by side
+  long long ch = blockIdx.x;
+  if (ch < C) {
+    const int c = (int)(ch / B), b = (int)(ch % B);
+    block_copy_async(vs, v + ((size_t)b * D + c) * (size_t)L, row_bytes, tl, TV);
+    block_copy_async(hs, pick(hh, 0) + (size_t)c * MV, h_bytes, tl, TV);
+    cp_async_commit();
+    cp_async_wait_all();
+  }
+  __syncthreads();
+
+  for (; ch < C; ch += gridDim.x) {
     const int c = (int)(ch / B), b = (int)(ch % B);
     const size_t row = ((size_t)b * D + c) * (size_t)L;
     float2 a[16];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int m = tl + r * Q16;
-      a[r] = (2 * m < L) ? IO<T>::load2_stream(v + row + 2 * m) : make_float2(0.f, 0.f);
+      a[r] = (2 * m < L) ? IO<T>::load2_smem(vs + 2 * m) : make_float2(0.f, 0.f);
     }
     for (int n = 0; n < N; ++n) {
       // forward: first pass (radix 16, upper half of the input is zero)
       dft16<false, true, false, 0>(a);
-#pragma unroll
-      for (int r = 0; r < 16; ++r) sm[pidx(16 * tl + r)] = a[r];
+      store_block16(sm, tl, a);
       __syncthreads();
+      // every thread is past its reads of the gate and v buffers: refill them
+      block_copy_async(xs, pick(x, n) + row, row_bytes, tl, TV);
+      if (n == 0 && ch + gridDim.x < C) {
+        const long long nx = ch + gridDim.x;
+        const int c2 = (int)(nx / B), b2 = (int)(nx % B);
+        block_copy_async(vs, v + ((size_t)b2 * D + c2) * (size_t)L, row_bytes, tl, TV);
+      }
+      cp_async_commit();
       mid_fwd_all<LOGMV>(a, sm, tw, tl);
-      // last forward pass + spectral product + first inverse pass
-      float2* H = const_cast<float2*>(pick(hh, n)) + (size_t)c * MV;
-      paired_pass<LOGMV, kPairConv>(sm, sm, jA, jB, head, tw, Wv, one, false, H, H, 0.f);
+      // spectrum of stage n, gate of stage n and the next v are resident after this barrier
+      cp_async_wait_all();
       __syncthreads();
+      // last forward pass + spectral product + first inverse pass
+      paired_pass<LOGMV, kPairConv, true>(sm, sm, jA, jB, head, tw, Wv, one, false, hs, hs, 0.f);
+      __syncthreads();
+      // the spectrum buffer is free: stage the next spectrum (next stage or next channel)
+      {
+        const float2* hn = nullptr;
+        if (n + 1 < N) {
+          hn = pick(hh, n + 1) + (size_t)c * MV;
+        } else if (ch + gridDim.x < C) {
+          hn = pick(hh, 0) + (size_t)((ch + gridDim.x) / B) * MV;
+        }
+        if (hn) block_copy_async(hs, hn, h_bytes, tl, TV);
+        cp_async_commit();
+      }
       mid_inv_all<LOGMV>(a, sm, tw, tl);
       // last inverse pass (radix 16): only the first half of the outputs is kept
-#pragma unroll
-      for (int r = 0; r < 16; ++r) a[r] = sm[pidx(16 * tl + r)];
+      load_block16(sm, tl, a);
       dft16<true, false, true, 0>(a);
       // gate: z_{n+1}[t] = x_n[t] * conv[t]
-      const T* __restrict__ xr = pick(x, n) + row;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int m = tl + r * Q16;
-        const float2 g = (2 * m < L) ? IO<T>::load2_stream(xr + 2 * m) : make_float2(0.f, 0.f);
+        const float2 g = (2 * m < L) ? IO<T>::load2_smem(xs + 2 * m) : make_float2(0.f, 0.f);
         a[r] = make_float2(a[r].x * g.x, a[r].y * g.y);
       }
     }
@@ -70,6 +126,7 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
       if (2 * m < L) IO<T>::store2(y + row + 2 * m, a[r]);
     }
   }
+  cp_async_wait_all();
 }
 
 // Filter spectrum for the fused layout: H[c][k] = rfft(pad(h_c, 2M))[k] / (4M)
@@ -80,7 +137,7 @@ fused_spectrum_kernel(const float* __restrict__ h, float2* __restrict__ spec, co
                       int D, int L) {
   using P = Plan<LOGMV>;
   constexpr int MV = P::MV, Q8 = MV / 8, Q16 = MV / 16;
-  extern __shared__ float2 sm[];
+  extern __shared__ __align__(16) float2 sm[];
   const int tl = threadIdx.x;
   const float2* __restrict__ tw = tables;
   const float2* __restrict__ Wv = tables + MV;
@@ -97,8 +154,7 @@ fused_spectrum_kernel(const float* __restrict__ h, float2* __restrict__ spec, co
       a[r] = (2 * m < L) ? __ldg(reinterpret_cast<const float2*>(hr + 2 * m)) : make_float2(0.f, 0.f);
     }
     dft16<false, true, false, 0>(a);
-#pragma unroll
-    for (int r = 0; r < 16; ++r) sm[pidx(16 * tl + r)] = a[r];
+    store_block16(sm, tl, a);
     __syncthreads();
     mid_fwd_all<LOGMV>(a, sm, tw, tl);
     float2* H = spec + (size_t)c * MV;
@@ -113,7 +169,7 @@ template <int LOGMV, typename T>
 static cudaError_t launch_fused_t(const FusedLaunch& p, cudaStream_t s) {
   auto k = fused_forward_kernel<LOGMV, T>;
   const int threads = Plan<LOGMV>::TV;
-  const size_t smem = sizeof(float2) * padded_len(1 << LOGMV);
+  const size_t smem = FusedSmem<LOGMV, T>::total;
   int grid = 0;
   cudaError_t e = persistent_grid((const void*)k, threads, smem, &grid);
   if (e != cudaSuccess) return e;

@@ -15,6 +15,19 @@ namespace hyena {
 
 enum PairMode { kPairConv = 0, kPairSpectrum = 1 };
 
+// Filter spectrum reads: from global memory through the read-only path, or
+// from a shared-memory copy staged by the caller (H_SMEM).
+template <bool H_SMEM>
+struct HRead;
+template <>
+struct HRead<false> {
+  static __device__ __forceinline__ float2 at(const float2* p, int i) { return __ldg(p + i); }
+};
+template <>
+struct HRead<true> {
+  static __device__ __forceinline__ float2 at(const float2* p, int i) { return p[i]; }
+};
+
 // W for bin kA of row A: w_{2M}^{k1 + M1 k2} = rho * w_{2 MV}^{k2}.
 __device__ __forceinline__ float2 pair_w(const float2* __restrict__ Wv, int k2, float2 rho, bool has_rho) {
   float2 w = __ldg(&Wv[k2]);
@@ -26,38 +39,28 @@ __device__ __forceinline__ float2 pair_w(const float2* __restrict__ Wv, int k2, 
 // MODE kPairSpectrum: the unpacked spectrum 2 Z[k] * scale is written to HA/HB
 //   (library order, packed DC/Nyquist in bin 0 of row 0); shared memory is not
 //   written back.
-template <int LOGMV, int MODE>
+template <int LOGMV, int MODE, bool H_SMEM = false>
 __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA, int jB, bool head,
                                             const float2* __restrict__ tw, const float2* __restrict__ Wv,
                                             float2 rho, bool has_rho, float2* HA, float2* HB, float scale) {
   constexpr int MV = 1 << LOGMV, Q8 = MV / 8, Q16 = MV / 16, NS = Q8;
+  auto hload = [](const float2* p, int i) { return HRead<H_SMEM>::at(p, i); };
   float2 a[8], b[8];
+  float2* pa = baseA + pidx(jA);
+  float2* pb = baseB + pidx(jB);
+  static_assert(Q8 % 16 == 0, "paired pass needs MV >= 128");
+  constexpr int QS = Q8 + Q8 / 16;   // padded stride between the bins of one butterfly
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    a[r] = baseA[pidx(jA + r * Q8)];
-    b[r] = baseB[pidx(jB + r * Q8)];
+    a[r] = pa[r * QS];
+    b[r] = pb[r * QS];
   }
-  // filter spectrum for the product (loaded early: independent of the FFT)
-  float2 ha[8], hb[8];
-  if (MODE == kPairConv) {
-    if (!head) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        ha[r] = __ldg(&HA[jA + r * Q8]);
-        hb[r] = __ldg(&HB[jB + (7 - r) * Q8]);
-      }
-    } else {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        ha[r] = __ldg(&HA[r * Q8]);
-        hb[r] = __ldg(&HA[Q16 + r * Q8]);
-      }
-    }
-  }
+  const float2* __restrict__ twa = tw + (NS - 1) + jA;
+  const float2* __restrict__ twb = tw + (NS - 1) + jB;
 #pragma unroll
   for (int r = 1; r < 8; ++r) {
-    a[r] = cmul(a[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jA]));
-    b[r] = cmul(b[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jB]));
+    a[r] = cmul(a[r], __ldg(twa + (r - 1) * NS));
+    b[r] = cmul(b[r], __ldg(twb + (r - 1) * NS));
   }
   dft8<false, 0>(a);
   dft8<false, 0>(b);
@@ -68,7 +71,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
       const int kA = jA + r * Q8;
       const float2 W = pair_w(Wv, kA, rho, has_rho);
       if (MODE == kPairConv) {
-        spectral_pair(a[r], b[7 - r], ha[r], hb[r], W);
+        spectral_pair(a[r], b[7 - r], hload(HA, kA), hload(HB, jB + (7 - r) * Q8), W);
       } else {
         float2 za, zb;
         unpack_pair(a[r], b[7 - r], W, za, zb);
@@ -83,7 +86,8 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
       const float2 one = make_float2(1.f, 0.f);
       if (MODE == kPairConv) {
         float2 c0 = a[0], c0b = a[0];
-        spectral_pair(c0, c0b, make_float2(ha[0].x, 0.f), make_float2(ha[0].y, 0.f), one);
+        const float2 h0 = hload(HA, 0);
+        spectral_pair(c0, c0b, make_float2(h0.x, 0.f), make_float2(h0.y, 0.f), one);
         a[0] = c0;
       } else {
         float2 za, zb;
@@ -95,7 +99,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     for (int r = 1; r < 4; ++r) {
       const float2 W = __ldg(&Wv[r * Q8]);
       if (MODE == kPairConv) {
-        spectral_pair(a[r], a[8 - r], ha[r], ha[8 - r], W);
+        spectral_pair(a[r], a[8 - r], hload(HA, r * Q8), hload(HA, (8 - r) * Q8), W);
       } else {
         float2 za, zb;
         unpack_pair(a[r], a[8 - r], W, za, zb);
@@ -107,7 +111,8 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
       const float2 W = __ldg(&Wv[4 * Q8]);
       if (MODE == kPairConv) {
         float2 c4 = a[4], c4b = a[4];
-        spectral_pair(c4, c4b, ha[4], ha[4], W);
+        const float2 h4 = hload(HA, 4 * Q8);
+        spectral_pair(c4, c4b, h4, h4, W);
         a[4] = c4;
       } else {
         float2 za, zb;
@@ -120,7 +125,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     for (int r = 0; r < 4; ++r) {
       const float2 W = __ldg(&Wv[Q16 + r * Q8]);
       if (MODE == kPairConv) {
-        spectral_pair(b[r], b[7 - r], hb[r], hb[7 - r], W);
+        spectral_pair(b[r], b[7 - r], hload(HA, Q16 + r * Q8), hload(HA, Q16 + (7 - r) * Q8), W);
       } else {
         float2 za, zb;
         unpack_pair(b[r], b[7 - r], W, za, zb);
@@ -135,13 +140,13 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     dft8<true, 0>(b);
 #pragma unroll
     for (int r = 1; r < 8; ++r) {
-      a[r] = cmulc(a[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jA]));
-      b[r] = cmulc(b[r], __ldg(&tw[NS - 1 + (r - 1) * NS + jB]));
+      a[r] = cmulc(a[r], __ldg(twa + (r - 1) * NS));
+      b[r] = cmulc(b[r], __ldg(twb + (r - 1) * NS));
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      baseA[pidx(jA + r * Q8)] = a[r];
-      baseB[pidx(jB + r * Q8)] = b[r];
+      pa[r * QS] = a[r];
+      pb[r * QS] = b[r];
     }
   }
 }
