@@ -126,11 +126,12 @@ hyena_status hyena_filter_rfft(const float* h, int D, int L, void* hhat, hyena_s
   if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
   float2* spec = reinterpret_cast<float2*>(hhat);
-  float2* tables = spec + (size_t)D * y.M;
+  float2* tables = spec + tables_offset(y, D);
   cudaError_t e = launch_fill_tables(tables, y, s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (!y.fourstep) {
     e = launch_fused_spectrum(h, spec, tables, D, L, y.logMV, s);
+    if (e == cudaSuccess && y.tc) e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(y, D), tables, D, y, s);
   } else {
     for (long long c0 = 0; c0 < D && e == cudaSuccess; c0 += kMaxGridY) {
       const int nd = (int)((D - c0) < kMaxGridY ? (D - c0) : kMaxGridY);
@@ -166,7 +167,7 @@ hyena_status hyena_forward(const void* v, const void* const* x, const void* cons
   Layout ly;
   if (!make_layout(L, &ly)) return HYENA_ERR_UNSUPPORTED;
   cudaStream_t s = (cudaStream_t)stream;
-  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + (size_t)D * ly.M;
+  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + tables_offset(ly, D);
   cudaError_t e = cudaSuccess;
   if (!ly.fourstep) {
     FusedLaunch p{};
@@ -179,7 +180,14 @@ hyena_status hyena_forward(const void* v, const void* const* x, const void* cons
     p.tables = tables;
     p.B = B; p.D = D; p.L = L; p.N = N;
     p.bf16 = (dtype == HYENA_BF16);
-    e = launch_fused_forward(p, ly.logMV, s);
+    if (ly.tc && p.bf16 && (B % 2) == 0) {
+      // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
+      for (int n = 0; n < N; ++n)
+        p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
+      e = launch_tc_forward(p, ly, s);
+    } else {
+      e = launch_fused_forward(p, ly.logMV, s);
+    }
   } else {
     const size_t per = sizeof(float2) * (size_t)ly.M;
     if (!aligned16(workspace) || workspace_bytes < per) return HYENA_ERR_WORKSPACE;

@@ -66,6 +66,9 @@ cudaError_t launch_fill_tables(float2* tables, const Layout& y, cudaStream_t s);
 cudaError_t launch_fused_forward(const FusedLaunch& p, int logMV, cudaStream_t s);
 cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* tables, int D, int L, int logMV,
                                   cudaStream_t s);
+cudaError_t launch_tc_forward(const FusedLaunch& p, const Layout& y, cudaStream_t s);
+cudaError_t launch_tc_spectrum(const float2* nat, float2* tcs, float2* tables, int D, const Layout& y,
+                               cudaStream_t s);
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
                                      const Layout& y, cudaStream_t s);

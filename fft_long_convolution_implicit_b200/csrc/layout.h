@@ -27,8 +27,16 @@ struct Layout {
   int tw_v;     // MV-point plan twiddles (MV entries)
   int w_v;      // w_{2 MV}^k, k < MV
   int tw_1;     // M1-point column plan twiddles (M1 entries, four-step only)
+  // tensor-core path (bf16, pairs of batch items): 2L = R0 * 256
+  bool tc;
+  int R0;
+  int tc_otw;   // outer twiddles w_{2L}^{m k0}, [k0 = 1..R0-1][m < 256] (R0 * 256 entries)
   int table_len;
 };
+
+// Lengths with a tensor-core forward (outer radix R0 = L / 128 in {8, 16}).
+constexpr int kTcMinL = 1024;
+constexpr int kTcMaxL = 2048;
 
 inline int ilog2_exact(int v) {
   int l = 0;
@@ -61,13 +69,24 @@ inline bool make_layout(int L, Layout* out) {
   y.w_v = y.MV;
   y.tw_1 = 2 * y.MV;
   y.table_len = 2 * y.MV + (y.fourstep ? y.M1 : 0);
+  y.tc = (L >= kTcMinL && L <= kTcMaxL);
+  y.R0 = y.tc ? L / 128 : 0;
+  y.tc_otw = y.table_len;
+  if (y.tc) y.table_len += y.R0 * 256;
   y.table_len = (y.table_len + 1) & ~1;   // keep the block a multiple of 16 bytes
   *out = y;
   return true;
 }
 
-// One filter's spectrum block: [D][M] float2 spectrum (library order) followed
-// by the table region.
-inline size_t spectrum_block_floats2(const Layout& y, int D) { return (size_t)D * y.M + y.table_len; }
+// One filter's spectrum block: [D][M] float2 spectrum (library order); for
+// tensor-core lengths a second copy [D][L] in the tensor-core order; then the
+// table region.
+// tensor-core copy: rows of L + 2 float2 (L bins, then (1/f_c, 0) and padding)
+inline int tc_row(const Layout& y) { return y.L + 2; }
+inline size_t tc_spectrum_offset(const Layout& y, int D) { return (size_t)D * y.M; }
+inline size_t tables_offset(const Layout& y, int D) {
+  return (size_t)D * y.M + (y.tc ? (size_t)D * tc_row(y) : 0);
+}
+inline size_t spectrum_block_floats2(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
 
 }  // namespace hyena

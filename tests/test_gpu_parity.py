@@ -88,6 +88,14 @@ SWEEP = [
     (2, "f32", 2, 1, 65536),
     (1, "f32", 1, 2, 262144),
     (2, "bf16", 1, 2, 524288),
+    # tensor-core kernel: bf16, even B, L in {1024, 2048}
+    (1, "bf16", 2, 3, 1024),
+    (2, "bf16", 2, 1, 2048),
+    (3, "bf16", 4, 5, 1024),
+    (4, "bf16", 2, 2, 2048),
+    (2, "bf16", 6, 3, 2048),
+    # odd B at a tensor-core length falls back to the SIMT kernel
+    (2, "bf16", 3, 2, 2048),
 ]
 
 
@@ -101,10 +109,10 @@ def test_forward_shapes(hy, N, dtype, B, D, L):
     assert err.max() <= TOL[dtype], err.max()
 
 
-@pytest.mark.parametrize("L", [2048, 32768])
-def test_forward_in_place_and_waves(hy, L):
+@pytest.mark.parametrize("L,dtype", [(2048, "f32"), (2048, "bf16"), (32768, "f32")])
+def test_forward_in_place_and_waves(hy, L, dtype):
     import torch
-    w = synth.custom(2, "f32", 2, 3, L, seed=5)
+    w = synth.custom(2, dtype, 2, 3, L, seed=5)
     y_ref, _, (v, xs, wt) = gpu_run(w)
     tw = weights_to_cuda(wt)
     h = hy.filter_generate(tw, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
@@ -114,11 +122,11 @@ def test_forward_in_place_and_waves(hy, L):
     txs = [upload(x, w) for x in xs]
     hy.forward(tv, txs, hh, y=tv)
     torch.cuda.synchronize()
-    np.testing.assert_array_equal(tv.cpu().numpy().reshape(w.channels, L), y_ref)
+    np.testing.assert_array_equal(tv.float().cpu().numpy().reshape(w.channels, L), y_ref)
     # y aliasing the last gate
     tv = upload(v, w)
     hy.forward(tv, txs, hh, y=txs[-1])
-    np.testing.assert_array_equal(txs[-1].cpu().numpy().reshape(w.channels, L), y_ref)
+    np.testing.assert_array_equal(txs[-1].float().cpu().numpy().reshape(w.channels, L), y_ref)
     if L > 8192:
         # a one-channel workspace: every channel runs in its own wave
         tv = upload(v, w)
@@ -150,9 +158,10 @@ def test_full_size_delta_filter_identity(hy, cfg_i):
     assert (num / den).max().item() <= TOL[w.dtype]
 
 
-def test_forward_is_deterministic_and_scales_exactly(hy):
+@pytest.mark.parametrize("cfg_i", [1, 2])
+def test_forward_is_deterministic_and_scales_exactly(hy, cfg_i):
     import torch
-    w = synth.workload(2)
+    w = synth.workload(cfg_i)
     g = torch.Generator(device="cuda").manual_seed(3)
     tv = torch.randn(w.B, w.D, w.L, device="cuda", generator=g).bfloat16()
     txs = [torch.randn(w.B, w.D, w.L, device="cuda", generator=g).bfloat16() for _ in range(w.N)]
