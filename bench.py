@@ -138,6 +138,29 @@ class ClockSampler:
                 "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
 
 
+# ------------------------------------------------------- replica helpers --
+
+def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
+    """Every rank processes its own batch of the same shape (weak scaling):
+    same workload, inputs seeded per rank."""
+    return synth.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(units_per_rank: float, world: int, elapsed_ms: float) -> float:
+    """Units processed by all ranks / max-over-ranks elapsed time, in 1e9 units/s."""
+    return units_per_rank * world / (elapsed_ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------- oracle arm --
 
 def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0):
@@ -229,7 +252,7 @@ def main():
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
 
     # inputs of this rank (seeded per rank), weights and cached spectra
-    wr = synth.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
+    wr = rank_workload(w, rank)
     v_np, xs_np = synth.inputs(wr)
     wt = synth.filter_weights(wr)
     tw = {k: torch.from_numpy(np.ascontiguousarray(a)).to(dev) for k, a in wt.items()}
@@ -284,13 +307,8 @@ def main():
     clocks = sampler.stop()
     elapsed_ms = start.elapsed_time(end)
     step_ms = [a.elapsed_time(b) for a, b in zip(ev_pre, ev_post)]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-
-    units = K * w.channels * w.L * world
-    value = units / (elapsed_ms * 1e-3) / 1e9
+    elapsed_ms = max_over_ranks(elapsed_ms, dist if world > 1 else None, dev)
+    value = whole_job_throughput(K * w.channels * w.L, world, elapsed_ms)
     kernel_ms = statistics.mean(step_ms)
     peak, peak_kind = hbm_peak()
     alg_bytes = w.roofline_bytes()
@@ -326,12 +344,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = args.e2e_steps * w.channels * w.L * world / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    e2e_value = whole_job_throughput(args.e2e_steps * w.channels * w.L, world, e2e_ms)
 
     line = None
     if rank == 0:
