@@ -48,7 +48,17 @@ L2_BYTES = 126 * 2 ** 20
 KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
+    "tc": ("tc_fused.cu", "fft_engine.cuh", "layout.h"),
 }
+
+
+def dominant_kernel(w: synth.Workload) -> tuple[str, str]:
+    """(kernel name, source set) of the launch that dominates one forward."""
+    if w.L > 8192:
+        return "four-step column/row kernels (whole step)", "fourstep"
+    if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
+        return "tc_forward_kernel", "tc"
+    return "fused_forward_kernel", "fused"
 
 
 def kernel_source_sha(path: str = "fused") -> str:
@@ -360,7 +370,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
                          "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
-                         "kernel": "fused_forward_kernel" if w.L <= 8192 else "whole step (four-step kernels)",
+                         "kernel": dominant_kernel(w)[0],
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
