@@ -60,7 +60,8 @@ cudaError_t hyena::persistent_grid(const void* kernel, int threads, size_t smem,
   int sms = 0;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  if (smem > 48 * 1024) {
+  // opt in whenever dynamic shared memory is used: static + dynamic may pass 48 KB
+  if (smem > 0) {
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
