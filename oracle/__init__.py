@@ -1,4 +1,4 @@
-"""float64 CPU oracle for the Hyena order-N forward (ctypes wrapper of oracle.c).
+"""float64 CPU oracle for the Hyena order-N forward and backward (ctypes wrapper of oracle.c).
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, by ``__graft_entry__.smoke()``
 and by the CPU-baseline leg of ``bench.py``. The CUDA library never imports
@@ -58,6 +58,13 @@ def lib():
                                     i32, P, P, P, i32]
         l.oracle_hyena_forward.argtypes = [P, P, P, P, i64, i32, i64, i32, P, i32]
         l.oracle_hyena_forward.restype = i32
+        for name in ("oracle_causal_corr_direct", "oracle_causal_corr_fft", "oracle_causal_corr",
+                     "oracle_causal_xcorr_direct", "oracle_causal_xcorr_fft", "oracle_causal_xcorr"):
+            getattr(l, name).argtypes = [P, P, i64, P]
+        l.oracle_hyena_backward.argtypes = [P, P, P, P, P, i64, i32, i64, i32, P, P, P, i32]
+        l.oracle_hyena_backward.restype = i32
+        l.oracle_filter_backward.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, d, d, P,
+                                             P, P, P, P, P, P, i32]
         _lib = l
     return _lib
 
@@ -158,3 +165,71 @@ def hyena_forward(v, xs, hs, filter_row=None, threads: int | None = None) -> np.
     if rc != 0:
         raise ValueError("oracle_hyena_forward rejected its arguments")
     return y
+
+
+def causal_corr(h, r, method: str = "auto") -> np.ndarray:
+    """Transpose of the causal sum: out[s] = sum_{t>=s} h[t-s] r[t], s < L."""
+    h, r = _f64(h), _f64(r)
+    assert h.shape == r.shape and h.ndim == 1
+    out = np.empty_like(r)
+    fn = {"auto": lib().oracle_causal_corr, "direct": lib().oracle_causal_corr_direct,
+          "fft": lib().oracle_causal_corr_fft}[method]
+    fn(_p(h), _p(r), len(r), _p(out))
+    return out
+
+
+def causal_xcorr(r, z, method: str = "auto") -> np.ndarray:
+    """Filter-gradient correlation: out[j] = sum_{t>=j} r[t] z[t-j], j < L."""
+    r, z = _f64(r), _f64(z)
+    assert r.shape == z.shape and r.ndim == 1
+    out = np.empty_like(r)
+    fn = {"auto": lib().oracle_causal_xcorr, "direct": lib().oracle_causal_xcorr_direct,
+          "fft": lib().oracle_causal_xcorr_fft}[method]
+    fn(_p(r), _p(z), len(r), _p(out))
+    return out
+
+
+def hyena_backward(v, xs, hs, dy, filter_row=None, threads: int | None = None):
+    """Gradients of <dy, y> through the order-N forward on independent channels.
+
+    v, dy: [C][L]; xs: N arrays [C][L]; hs: N arrays [F][L]; filter_row as in
+    hyena_forward. Returns (dv [C][L], dx [N][C][L], dh [N][F][L]) where dh sums
+    the contributions of every channel that uses a filter row.
+    """
+    v = _f64(np.atleast_2d(v))
+    C, L = v.shape
+    N = len(xs)
+    x = _f64(np.stack([np.atleast_2d(a) for a in xs]))
+    h = _f64(np.stack([np.atleast_2d(a) for a in hs]))
+    dy = _f64(np.atleast_2d(dy))
+    assert x.shape == (N, C, L) and h.shape[0] == N and h.shape[2] == L and dy.shape == (C, L)
+    F = h.shape[1]
+    fr = np.ascontiguousarray(np.arange(C) if filter_row is None else filter_row, dtype=np.int32)
+    assert fr.shape == (C,) and (fr >= 0).all() and (fr < F).all()
+    dv = np.empty((C, L))
+    dx = np.empty((N, C, L))
+    dh_ch = np.empty((N, C, L))
+    rc = lib().oracle_hyena_backward(_p(v), _p(x), _p(h), _p(dy), _p(fr), C, F, L, N,
+                                     _p(dv), _p(dx), _p(dh_ch), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_hyena_backward rejected its arguments")
+    dh = np.zeros((N, F, L))
+    for r in range(C):
+        dh[:, fr[r], :] += dh_ch[:, r, :]
+    return dv, dx, dh
+
+
+def filter_backward(weights: dict, N: int, D: int, L: int, alpha_lo: float, alpha_hi: float, dh,
+                    n_bands: int = 8, threads: int | None = None) -> dict:
+    """Gradients of <dh, h> w.r.t. the implicit-filter weights (float64 dict
+    with keys W1, b1, W2, b2, W3, b3). dh: [N][D][L] or [N*D][L]."""
+    W1, b1, W2, b2, W3, b3 = (_f32(weights[k]) for k in ("W1", "b1", "W2", "b2", "W3", "b3"))
+    width = W1.shape[0]
+    dh = _f64(np.asarray(dh).reshape(N * D, L))
+    out = {"W1": np.empty(W1.shape), "b1": np.empty(b1.shape), "W2": np.empty(W2.shape),
+           "b2": np.empty(b2.shape), "W3": np.empty(W3.shape), "b3": np.empty(b3.shape)}
+    lib().oracle_filter_backward(_p(W1), _p(b1), _p(W2), _p(b2), _p(W3), _p(b3), n_bands, width,
+                                 N, D, L, float(alpha_lo), float(alpha_hi), _p(dh),
+                                 *(_p(out[k]) for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
+                                 threads or default_threads())
+    return out
