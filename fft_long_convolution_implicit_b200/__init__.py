@@ -1,4 +1,4 @@
-"""Hyena order-N forward on B200 (sm_100a): thin Python binding of libhyena_b200.so.
+"""Hyena order-N forward and backward on B200 (sm_100a): thin Python binding of libhyena_b200.so.
 
 Every function here marshals arguments (torch CUDA tensors -> device
 pointers, the current CUDA stream) and calls the C ABI declared in
@@ -9,6 +9,8 @@ an exception is raised.
     h    = filter_generate(weights, N, D, L, alpha_lo, alpha_hi)      # [N][D][L] fp32
     hhat = [filter_rfft(h[n]) for n in range(N)]                      # cached spectra
     y    = forward(v, [x1, ..., xN], hhat)                            # [B][D][L]
+    dv, dxs, dh = backward(v, [x1, ..., xN], hhat, dy)                # gradients
+    grads = filter_backward(weights, N, D, L, alpha_lo, alpha_hi, dh) # FFN weight gradients
 """
 from __future__ import annotations
 
@@ -25,7 +27,8 @@ HYENA_F32, HYENA_BF16 = 0, 1
 EXPORTS = (
     "hyena_filter_generate", "hyena_filter_spectrum_bytes", "hyena_filter_rfft", "hyena_spectrum_layout",
     "hyena_forward_workspace_bytes", "hyena_forward", "hyena_status_string", "hyena_last_cuda_error",
-    "hyena_abi_version", "hyena_forward_static_workspace",
+    "hyena_abi_version", "hyena_forward_static_workspace", "hyena_backward_workspace_bytes", "hyena_backward",
+    "hyena_filter_backward_workspace_bytes", "hyena_filter_backward",
 )
 
 
@@ -37,6 +40,11 @@ class HyenaError(RuntimeError):
             msg += ": " + lib.hyena_last_cuda_error().decode()
         super().__init__(f"{where}: {msg}")
         self.status = status
+
+
+class FilterGrads(ctypes.Structure):
+    _fields_ = [("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p), ("W2", ctypes.c_void_p),
+                ("b2", ctypes.c_void_p), ("W3", ctypes.c_void_p), ("b3", ctypes.c_void_p)]
 
 
 class FilterParams(ctypes.Structure):
@@ -72,6 +80,15 @@ def load() -> ctypes.CDLL:
     l.hyena_forward.restype = i
     l.hyena_forward_static_workspace.argtypes = [P, P, P, i, i, i, i, i, P, P]
     l.hyena_forward_static_workspace.restype = i
+    l.hyena_backward_workspace_bytes.argtypes = [i, i, i, i, i]
+    l.hyena_backward_workspace_bytes.restype = sz
+    l.hyena_backward.argtypes = [P, P, P, P, i, i, i, i, i, P, P, P, P, sz, P]
+    l.hyena_backward.restype = i
+    l.hyena_filter_backward_workspace_bytes.argtypes = [i, i, i, i, i]
+    l.hyena_filter_backward_workspace_bytes.restype = sz
+    l.hyena_filter_backward.argtypes = [ctypes.POINTER(FilterParams), i, i, i, ctypes.c_float, ctypes.c_float, P,
+                                        ctypes.POINTER(FilterGrads), P, sz, P]
+    l.hyena_filter_backward.restype = i
     l.hyena_status_string.argtypes = [i]
     l.hyena_status_string.restype = ctypes.c_char_p
     l.hyena_last_cuda_error.argtypes = []
@@ -125,6 +142,14 @@ def filter_spectrum_bytes(D: int, L: int) -> int:
 
 def forward_workspace_bytes(B: int, D: int, L: int, N: int, bf16: bool) -> int:
     return load().hyena_forward_workspace_bytes(B, D, L, N, HYENA_BF16 if bf16 else HYENA_F32)
+
+
+def backward_workspace_bytes(B: int, D: int, L: int, N: int, bf16: bool) -> int:
+    return load().hyena_backward_workspace_bytes(B, D, L, N, HYENA_BF16 if bf16 else HYENA_F32)
+
+
+def filter_backward_workspace_bytes(N: int, D: int, L: int, n_bands: int = 8, width: int = 64) -> int:
+    return load().hyena_filter_backward_workspace_bytes(N, D, L, n_bands, width)
 
 
 def spectrum_layout(L: int) -> tuple[int, int, int]:
@@ -211,6 +236,61 @@ def forward_static_workspace(v, xs, hhats, y=None, stream=None):
     _check(load().hyena_forward_static_workspace(_dev(v, "v"), xarr, harr, B, D, L, N, code, _dev(y, "y"),
                                                  _stream(stream)), "hyena_forward_static_workspace")
     return y
+
+
+def backward(v, xs, hhats, dy, dv=None, dxs=None, dh=None, workspace=None, stream=None):
+    """Gradients of <dy, y> for y = forward(v, xs, hhats): returns (dv, dxs, dh)
+    with dv and dxs[n] like v, and dh float32 [N][D][L] (filter gradients
+    summed over the batch)."""
+    torch = _torch()
+    B, D, L = v.shape
+    N = len(xs)
+    if len(hhats) != N:
+        raise ValueError("need one spectrum per gate")
+    code = _dtype_code(v)
+    for t in list(xs) + [dy]:
+        if t.shape != v.shape or t.dtype != v.dtype:
+            raise ValueError("gates and dy must match v in shape and dtype")
+    dv = torch.empty_like(v) if dv is None else dv
+    dxs = [torch.empty_like(v) for _ in range(N)] if dxs is None else list(dxs)
+    dh = torch.empty((N, D, L), dtype=torch.float32, device=v.device) if dh is None else dh
+    need = backward_workspace_bytes(B, D, L, N, code == HYENA_BF16)
+    if need == 0:
+        _check(HYENA_ERR_INVALID_ARG, "hyena_backward_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    xarr = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+    harr = (ctypes.c_void_p * N)(*[_dev(hh, "hhat").value for hh in hhats])
+    dxarr = (ctypes.c_void_p * N)(*[_dev(t, "dx").value for t in dxs])
+    dharr = (ctypes.c_void_p * N)(*[_dev(dh[n], "dh").value for n in range(N)])
+    _check(load().hyena_backward(_dev(v, "v"), xarr, harr, _dev(dy, "dy"), B, D, L, N, code, _dev(dv, "dv"),
+                                 dxarr, dharr, _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)), "hyena_backward")
+    return dv, dxs, dh
+
+
+def filter_backward(weights: dict, N: int, D: int, L: int, alpha_lo: float, alpha_hi: float, dh,
+                    n_bands: int = 8, grads=None, workspace=None, stream=None) -> dict:
+    """Gradients of sum(dh * h) w.r.t. the FFN weights (float32 CUDA tensors
+    shaped like the weights). dh: float32 [N][D][L]."""
+    torch = _torch()
+    W1 = weights["W1"]
+    keys = ("W1", "b1", "W2", "b2", "W3", "b3")
+    if grads is None:
+        grads = {k: torch.empty_like(weights[k]) for k in keys}
+    width = W1.shape[0]
+    need = filter_backward_workspace_bytes(N, D, L, n_bands, width)
+    if need == 0:
+        _check(HYENA_ERR_INVALID_ARG, "hyena_filter_backward_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W1.device)
+    p = FilterParams(*(ctypes.c_void_p(_dev(weights[k], k).value) for k in keys), n_bands, width)
+    g = FilterGrads(*(ctypes.c_void_p(_dev(grads[k], "grad " + k).value) for k in keys))
+    _check(load().hyena_filter_backward(ctypes.byref(p), N, D, L, alpha_lo, alpha_hi, _dev(dh, "dh"),
+                                        ctypes.byref(g), _dev(workspace, "workspace"),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "hyena_filter_backward")
+    return grads
 
 
 def spectrum_natural(hhat, D: int, L: int):

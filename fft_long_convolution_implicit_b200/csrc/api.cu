@@ -75,6 +75,84 @@ cudaError_t hyena::persistent_grid(const void* kernel, int threads, size_t smem,
   return cudaSuccess;
 }
 
+cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const void* const* hhat, int B, int D,
+                                    const Layout& ly, int N, bool bf16, void* y, void* workspace,
+                                    size_t workspace_bytes, bool allow_tc, cudaStream_t s) {
+  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + tables_offset(ly, D);
+  cudaError_t e = cudaSuccess;
+  if (!ly.fourstep) {
+    FusedLaunch p{};
+    p.v = v;
+    for (int n = 0; n < N; ++n) {
+      p.x[n] = x[n];
+      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
+    }
+    p.y = y;
+    p.tables = tables;
+    p.B = B; p.D = D; p.L = ly.L; p.N = N;
+    p.bf16 = bf16;
+    if (allow_tc && ly.tc && p.bf16 && (B % 2) == 0) {
+      // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
+      for (int n = 0; n < N; ++n)
+        p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
+      e = launch_tc_forward(p, ly, s);
+    } else {
+      e = launch_fused_forward(p, ly.logMV, s);
+    }
+  } else {
+    const size_t per = sizeof(float2) * (size_t)ly.M;
+    const long long C = (long long)B * D;
+    long long w = (long long)(workspace_bytes / per);
+    if (w < 1) return cudaErrorInvalidValue;
+    if (w > C) w = C;
+    if (w > kMaxGridY) w = kMaxGridY;
+    FourStepLaunch p{};
+    p.v = v;
+    for (int n = 0; n < N; ++n) {
+      p.x[n] = x[n];
+      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
+    }
+    p.y = y;
+    p.tables = tables;
+    p.scratch = reinterpret_cast<float2*>(workspace);
+    p.B = B; p.D = D; p.L = ly.L; p.N = N;
+    p.bf16 = bf16;
+    for (long long c0 = 0; c0 < C && e == cudaSuccess; c0 += w) {
+      p.ch0 = c0;
+      p.wave = (int)((C - c0) < w ? (C - c0) : w);
+      e = launch_fourstep_wave(p, ly, s);
+    }
+  }
+  return e;
+}
+
+size_t hyena::fourstep_wave_bytes(long long channels, const Layout& ly) {
+  const size_t per = sizeof(float2) * (size_t)ly.M;
+  long long w = (long long)(kWaveTargetBytes / per);
+  if (w < 1) w = 1;
+  if (w > channels) w = channels;
+  if (w > kMaxGridY) w = kMaxGridY;
+  return per * (size_t)w;
+}
+
+cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, const Layout& ly, bool with_tc,
+                                     cudaStream_t s) {
+  float2* tables = spec + tables_offset(ly, rows);
+  cudaError_t e = launch_fill_tables(tables, ly, s);
+  if (e != cudaSuccess) return e;
+  if (!ly.fourstep) {
+    e = launch_fused_spectrum(h, spec, tables, rows, ly.L, ly.logMV, s);
+    if (e == cudaSuccess && with_tc && ly.tc)
+      e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
+  } else {
+    for (long long c0 = 0; c0 < rows && e == cudaSuccess; c0 += kMaxGridY) {
+      const int nd = (int)((rows - c0) < kMaxGridY ? (rows - c0) : kMaxGridY);
+      e = launch_fourstep_spectrum(h + (size_t)c0 * ly.L, spec + (size_t)c0 * ly.M, tables, nd, ly, s);
+    }
+  }
+  return e;
+}
+
 extern "C" {
 
 int hyena_abi_version(void) { return HYENA_ABI_VERSION; }
@@ -125,20 +203,7 @@ hyena_status hyena_filter_rfft(const float* h, int D, int L, void* hhat, hyena_s
   if (!aligned16(h) || !aligned16(hhat) || D < 1) return HYENA_ERR_INVALID_ARG;
   Layout y;
   if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
-  cudaStream_t s = (cudaStream_t)stream;
-  float2* spec = reinterpret_cast<float2*>(hhat);
-  float2* tables = spec + tables_offset(y, D);
-  cudaError_t e = launch_fill_tables(tables, y, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  if (!y.fourstep) {
-    e = launch_fused_spectrum(h, spec, tables, D, L, y.logMV, s);
-    if (e == cudaSuccess && y.tc) e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(y, D), tables, D, y, s);
-  } else {
-    for (long long c0 = 0; c0 < D && e == cudaSuccess; c0 += kMaxGridY) {
-      const int nd = (int)((D - c0) < kMaxGridY ? (D - c0) : kMaxGridY);
-      e = launch_fourstep_spectrum(h + (size_t)c0 * L, spec + (size_t)c0 * y.M, tables, nd, y, s);
-    }
-  }
+  const cudaError_t e = spectrum_dispatch(h, reinterpret_cast<float2*>(hhat), D, y, true, (cudaStream_t)stream);
   return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
 }
 
@@ -147,13 +212,7 @@ size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dty
   if (B < 1 || D < 1 || N < 1 || N > kMaxOrder || (dtype != HYENA_F32 && dtype != HYENA_BF16)) return 0;
   if (!make_layout(L, &y)) return 0;
   if (!y.fourstep) return 0;
-  const size_t per = sizeof(float2) * (size_t)y.M;
-  long long w = (long long)(kWaveTargetBytes / per);
-  if (w < 1) w = 1;
-  const long long C = (long long)B * D;
-  if (w > C) w = C;
-  if (w > kMaxGridY) w = kMaxGridY;
-  return per * (size_t)w;
+  return fourstep_wave_bytes((long long)B * D, y);
 }
 
 hyena_status hyena_forward(const void* v, const void* const* x, const void* const* hhat, int B, int D, int L,
@@ -167,52 +226,10 @@ hyena_status hyena_forward(const void* v, const void* const* x, const void* cons
   if ((long long)B * D > (1LL << 40) / (L > 0 ? L : 1)) return HYENA_ERR_INVALID_ARG;
   Layout ly;
   if (!make_layout(L, &ly)) return HYENA_ERR_UNSUPPORTED;
-  cudaStream_t s = (cudaStream_t)stream;
-  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + tables_offset(ly, D);
-  cudaError_t e = cudaSuccess;
-  if (!ly.fourstep) {
-    FusedLaunch p{};
-    p.v = v;
-    for (int n = 0; n < N; ++n) {
-      p.x[n] = x[n];
-      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
-    }
-    p.y = y;
-    p.tables = tables;
-    p.B = B; p.D = D; p.L = L; p.N = N;
-    p.bf16 = (dtype == HYENA_BF16);
-    if (ly.tc && p.bf16 && (B % 2) == 0) {
-      // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
-      for (int n = 0; n < N; ++n)
-        p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
-      e = launch_tc_forward(p, ly, s);
-    } else {
-      e = launch_fused_forward(p, ly.logMV, s);
-    }
-  } else {
-    const size_t per = sizeof(float2) * (size_t)ly.M;
-    if (!aligned16(workspace) || workspace_bytes < per) return HYENA_ERR_WORKSPACE;
-    const long long C = (long long)B * D;
-    long long w = (long long)(workspace_bytes / per);
-    if (w > C) w = C;
-    if (w > kMaxGridY) w = kMaxGridY;
-    FourStepLaunch p{};
-    p.v = v;
-    for (int n = 0; n < N; ++n) {
-      p.x[n] = x[n];
-      p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]);
-    }
-    p.y = y;
-    p.tables = tables;
-    p.scratch = reinterpret_cast<float2*>(workspace);
-    p.B = B; p.D = D; p.L = L; p.N = N;
-    p.bf16 = (dtype == HYENA_BF16);
-    for (long long c0 = 0; c0 < C && e == cudaSuccess; c0 += w) {
-      p.ch0 = c0;
-      p.wave = (int)((C - c0) < w ? (C - c0) : w);
-      e = launch_fourstep_wave(p, ly, s);
-    }
-  }
+  if (ly.fourstep && (!aligned16(workspace) || workspace_bytes < sizeof(float2) * (size_t)ly.M))
+    return HYENA_ERR_WORKSPACE;
+  const cudaError_t e = forward_dispatch(v, x, hhat, B, D, ly, N, dtype == HYENA_BF16, y, workspace,
+                                         workspace_bytes, true, (cudaStream_t)stream);
   return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
 }
 

@@ -59,6 +59,19 @@ struct FourStepLaunch {
 // returns HYENA_ERR_CUDA.
 hyena_status report_cuda_error(cudaError_t e);
 
+// The forward on any supported layout: fused kernel (tensor-core kernel for
+// bf16 pairs when allow_tc), or four-step waves through the workspace.
+// Arguments are assumed checked by the caller.
+cudaError_t forward_dispatch(const void* v, const void* const* x, const void* const* hhat, int B, int D,
+                             const Layout& ly, int N, bool bf16, void* y, void* workspace, size_t workspace_bytes,
+                             bool allow_tc, cudaStream_t s);
+// Workspace of one L2-sized four-step wave over `channels` channels.
+size_t fourstep_wave_bytes(long long channels, const Layout& ly);
+// Spectrum block (spectra, optional tensor-core copy, tables) of `rows` real
+// rows h [rows][L] float32.
+cudaError_t spectrum_dispatch(const float* h, float2* spec, int rows, const Layout& ly, bool with_tc,
+                              cudaStream_t s);
+
 // Grid for a persistent kernel: SM count x resident CTAs per SM.
 cudaError_t persistent_grid(const void* kernel, int threads, size_t smem, int* grid);
 

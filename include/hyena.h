@@ -1,5 +1,5 @@
 /*
- * hyena.h -- C ABI of the B200 (sm_100a) Hyena order-N forward library.
+ * hyena.h -- C ABI of the B200 (sm_100a) Hyena order-N forward/backward library.
  *
  * The operator (order-N recurrence; "Hyena Hierarchy - Towards Larger
  * Convolutional Language Models" digest, section 방법 (Method) / 프레임워크
@@ -41,7 +41,7 @@
 extern "C" {
 #endif
 
-#define HYENA_ABI_VERSION 1
+#define HYENA_ABI_VERSION 2
 
 typedef enum {
   HYENA_OK = 0,
@@ -165,6 +165,64 @@ hyena_status hyena_forward(const void *v, const void *const *x, const void *cons
 #define HYENA_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
 hyena_status hyena_forward_static_workspace(const void *v, const void *const *x, const void *const *hhat, int B,
                                             int D, int L, int N, hyena_dtype dtype, void *y, hyena_stream stream);
+
+/*
+ * Gradients (no counterpart printed on the pages, which only mention training
+ * at 1M tokens: glossary "Hyena（ハイエナ）", section 応用). They are the chain
+ * rule through the definitions above:
+ *   u_n = h_n * z_n,  z_{n+1} = x_n (.) u_n,  g_{N+1} = dy,  r_n = g_{n+1} (.) x_n
+ *   dx_n       = g_{n+1} (.) u_n
+ *   g_n[s]     = sum_{t>=s} h_n[t-s] r_n[t]             (transpose of the causal sum)
+ *   dh_n[c][j] = sum_b sum_{t>=j} r_n[b][c][t] z_n[b][c][t-j]
+ *   dv         = g_1
+ * Both correlations are causal convolutions of time-reversed rows and run on
+ * the forward's 2L-grid FFT kernels in float32.
+ */
+
+/* Workspace bytes hyena_backward needs for this shape (0 when invalid):
+ * about (N + 5) * 4 * B*D*L + 24 * B*D*L + 8 * D*L bytes. */
+size_t hyena_backward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dtype);
+
+/*
+ * hyena_backward -- dv, dx_n and dh_n for the loss gradient dy = dL/dy of
+ * y = hyena_forward(v, x, hhat).
+ *   v, x, hhat, B, D, L, N, dtype: exactly as given to hyena_forward
+ *   dy:  device [B][D][L] dtype
+ *   dv:  device [B][D][L] dtype
+ *   dx:  host array of N device pointers, dx[n] = dL/dx_{n+1}, [B][D][L] dtype
+ *   dh:  host array of N device pointers, dh[n] = dL/dh_{n+1}, float32 [D][L]
+ *        (time-domain filter gradient, summed over the batch; the layout of
+ *        hyena_filter_generate's output, so dh[n] may point at h_grad + n*D*L)
+ *   workspace: device scratch of at least hyena_backward_workspace_bytes()
+ *        (HYENA_ERR_WORKSPACE otherwise). Outputs must not alias inputs or
+ *        the workspace.
+ */
+hyena_status hyena_backward(const void *v, const void *const *x, const void *const *hhat, const void *dy, int B,
+                            int D, int L, int N, hyena_dtype dtype, void *dv, void *const *dx, float *const *dh,
+                            void *workspace, size_t workspace_bytes, hyena_stream stream);
+
+/* Gradients of the implicit-filter weights: device float32 arrays shaped
+ * like the fields of hyena_filter_params; every element is overwritten. */
+typedef struct {
+  float *W1, *b1, *W2, *b2, *W3, *b3;
+} hyena_filter_grads;
+
+/* Workspace bytes hyena_filter_backward needs (0 when invalid). */
+size_t hyena_filter_backward_workspace_bytes(int N, int D, int L, int n_bands, int width);
+
+/*
+ * hyena_filter_backward -- gradients of sum_{n,c,t} dh[n][c][t] h[n][c][t]
+ * with respect to the FFN weights of hyena_filter_generate, by the chain rule
+ * through h = window (W3 s2 + b3), s2 = sin(W2 s1 + b2), s1 = sin(W1 e + b1):
+ *   dO = dh * window;  dW3 = sum_t dO s2^T,  db3 = sum_t dO
+ *   dp2 = cos(W2 s1 + b2) (.) W3^T dO;  dW2 = sum_t dp2 s1^T,  db2 = sum_t dp2
+ *   dp1 = cos(W1 e + b1) (.) W2^T dp2;  dW1 = sum_t dp1 e^T,   db1 = sum_t dp1
+ * dh: device float32 [N][D][L] (e.g. hyena_backward's dh outputs laid end to
+ * end). Sums over taps run in float32 in fixed chunks (deterministic).
+ */
+hyena_status hyena_filter_backward(const hyena_filter_params *p, int N, int D, int L, float alpha_lo,
+                                   float alpha_hi, const float *dh, const hyena_filter_grads *g, void *workspace,
+                                   size_t workspace_bytes, hyena_stream stream);
 
 /* Static description of a status code. */
 const char *hyena_status_string(hyena_status s);

@@ -17,7 +17,9 @@ tensor can be regenerated on its own:
   counter indices ``2 i`` and ``2 i + 1``.
 
 Tensor ids: 0 = v, n = x_n (n = 1..N), 101..106 = W1, b1, W2, b2, W3, b3,
-200 = the 4 x D embedding table E, 201 = the symbol stream.
+200 = the 4 x D embedding table E, 201 = the symbol stream, 300 = the loss
+gradient dy fed to the backward, 301 = a filter gradient dh fed to the
+filter-weight backward on its own.
 """
 from __future__ import annotations
 
@@ -36,6 +38,8 @@ TID_V = 0
 TID_W1, TID_B1, TID_W2, TID_B2, TID_W3, TID_B3 = 101, 102, 103, 104, 105, 106
 TID_EMBED = 200
 TID_SYMBOLS = 201
+TID_DY = 300
+TID_DH = 301
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -228,6 +232,16 @@ def inputs(w: Workload, rows: list[int] | None = None) -> tuple[np.ndarray, list
     """(v, [x_1..x_N]) as float32 arrays of shape [len(rows)][L]
     (all channels in b-major order when rows is None)."""
     return v_rows(w, rows), [x_rows(w, n, rows) for n in range(1, w.N + 1)]
+
+
+def dy_rows(w: Workload, rows: list[int] | None = None) -> np.ndarray:
+    """Loss gradient dL/dy [len(rows)][L]: N(0,1) in the storage type."""
+    return _rows(w, TID_DY, rows, "normal")
+
+
+def dh_rows(w: Workload) -> np.ndarray:
+    """A filter gradient dL/dh, float32 [N][D][L] of N(0,1) values."""
+    return normal(w.seed, TID_DH, 0, w.N * w.D * w.L).astype(np.float32).reshape(w.N, w.D, w.L)
 
 
 def sample_rows(w: Workload, count: int, salt: int = 0) -> list[int]:

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_host_queries(lib):
-    assert hy.abi_version() == 1
+    assert hy.abi_version() == 2
     assert lib.hyena_status_string(0) == b"ok"
     # spectrum block: D*M complex64 + tables
     M, M1, MV = hy.spectrum_layout(2048)
@@ -93,3 +93,33 @@ def test_status_strings(lib):
     for s in range(5):
         assert lib.hyena_status_string(s)
     assert lib.hyena_last_cuda_error() == b""
+
+
+def test_backward_queries_and_host_rejections(lib):
+    ws = hy.backward_workspace_bytes(2, 3, 1024, 2, False)
+    # u_1..u_N, z and rev(r), g, unit gates: (N + 4) float32 tensors, plus spectra of 2BD rows
+    assert ws >= (2 + 4) * 4 * 2 * 3 * 1024 + 2 * 2 * 3 * 1024 * 8
+    assert hy.backward_workspace_bytes(2, 3, 1000, 2, False) == 0
+    assert hy.backward_workspace_bytes(2, 3, 1024, 9, False) == 0
+    assert hy.filter_backward_workspace_bytes(2, 16, 1024) > 0
+    assert hy.filter_backward_workspace_bytes(2, 16, 1000) == 0
+    p = ctypes.c_void_p(16)
+    xs = (ctypes.c_void_p * 2)(16, 16)
+    f = lib.hyena_backward
+    # unsupported length, bad order, null arrays, misaligned pointer, small workspace
+    assert f(p, xs, xs, p, 1, 1, 1000, 2, 0, p, xs, xs, p, 1 << 30, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert f(p, xs, xs, p, 1, 1, 1024, 0, 0, p, xs, xs, p, 1 << 30, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, p, 1, 1, 1024, 2, 0, p, None, xs, p, 1 << 30, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, ctypes.c_void_p(24), 1, 1, 1024, 2, 0, p, xs, xs, p, 1 << 30, None) == hy.HYENA_ERR_INVALID_ARG
+    need = hy.backward_workspace_bytes(1, 1, 1024, 2, False)
+    assert f(p, xs, xs, p, 1, 1, 1024, 2, 0, p, xs, xs, p, need - 1, None) == hy.HYENA_ERR_WORKSPACE
+    assert f(p, xs, xs, p, 1, 1, 1024, 2, 0, p, xs, xs, None, need, None) == hy.HYENA_ERR_WORKSPACE
+    fp = hy.FilterParams(16, 16, 16, 16, 16, 16, 8, 64)
+    g = hy.FilterGrads(16, 16, 16, 16, 16, 16)
+    fb = lib.hyena_filter_backward
+    need = hy.filter_backward_workspace_bytes(2, 4, 256)
+    assert fb(ctypes.byref(fp), 2, 4, 256, 0.5, 20.0, p, ctypes.byref(g), p, need - 1, None) == hy.HYENA_ERR_WORKSPACE
+    assert fb(ctypes.byref(fp), 2, 4, 300, 0.5, 20.0, p, ctypes.byref(g), p, need, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert fb(None, 2, 4, 256, 0.5, 20.0, p, ctypes.byref(g), p, need, None) == hy.HYENA_ERR_INVALID_ARG
+    bad = hy.FilterGrads(16, 16, 16, 16, None, 16)
+    assert fb(ctypes.byref(fp), 2, 4, 256, 0.5, 20.0, p, ctypes.byref(bad), p, need, None) == hy.HYENA_ERR_INVALID_ARG
