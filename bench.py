@@ -2,6 +2,7 @@
 """Benchmark of the Hyena order-N forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config I]
+                    [--pass forward|backward]
 
 A step is one hyena_forward over one batch of the workload (default: the
 order-2, bf16, B=4, D=768, L=2048 workload), with the filter spectra already
@@ -14,6 +15,10 @@ and the fraction of the HBM roofline; one JSON line is printed by rank 0.
 (weak scaling, no collective on the data path); time is the max over ranks.
 --impl reference times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only).
+--pass backward times hyena_backward instead (dv, dx_n and dh_n from a loss
+gradient dy), same workload and conventions; its roofline counts the bytes
+the gradients must move at least: v, x_n, dy and the spectra in, dv, dx_n
+and dh_n out.
 """
 from __future__ import annotations
 
@@ -36,6 +41,7 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 METRIC = "Hyena order-N fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
+METRIC_BWD = "Hyena order-N bwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
 UNIT = "1e9 B*D*L/s"
 KERNEL_SOURCES = os.path.join(ROOT, "fft_long_convolution_implicit_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -59,6 +65,36 @@ def dominant_kernel(w: synth.Workload) -> tuple[str, str]:
     if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
         return "tc_forward_kernel", "tc"
     return "fused_forward_kernel", "fused"
+
+
+def backward_bytes(w: synth.Workload) -> int:
+    """Algorithmic bytes of one backward: v, x_1..x_N and dy read, dv and
+    dx_1..x_N written (storage type), the N spectra read (8 B per bin, as in
+    the forward), the N float32 filter gradients written."""
+    return ((2 * w.N + 3) * w.channels * w.L * w.elem_bytes + w.N * w.D * (w.L + 1) * 8
+            + 4 * w.N * w.D * w.L)
+
+
+def count_kernel_nodes(make_call) -> int:
+    """Kernels one call launches: capture it (on a side stream) into a CUDA
+    graph and count the kernel nodes."""
+    import torch
+    import cuda.bindings.runtime as rt
+    side = torch.cuda.Stream()
+    fn = make_call(side)
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        fn()
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    err, _, n = rt.cudaGraphGetNodes(graph, 0)
+    err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    count = sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+    g.reset()
+    return count
 
 
 def kernel_source_sha(path: str = "fused") -> str:
@@ -173,36 +209,36 @@ def whole_job_throughput(units_per_rank: float, world: int, elapsed_ms: float) -
 
 # ----------------------------------------------------------- oracle arm --
 
-def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0):
+def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0, backward: bool = False):
     """Time the float64 oracle (as it stands) on a bounded sample of rows of
     the workload; filters are computed beforehand and not timed."""
     import oracle
     threads = host_cores()
     wt = synth.filter_weights(w)
-    # calibrate: one row, then size the sample for ~target core-seconds
-    probe_rows = [0]
-    v, xs = synth.inputs(w, probe_rows)
-    cs = [0]
-    hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
-                                   rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
-    hs = [hrows[n:n + 1] for n in range(w.N)]
-    t0 = time.perf_counter()
-    oracle.hyena_forward(v, xs, hs, threads=1)
-    per_row = max(time.perf_counter() - t0, 1e-4)
+
+    def run(rows, n_threads):
+        v, xs = synth.inputs(w, rows)
+        cs = sorted({r % w.D for r in rows})
+        hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
+                                       rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
+        hs = [hrows[n * len(cs):(n + 1) * len(cs)] for n in range(w.N)]
+        fr = [cs.index(r % w.D) for r in rows]
+        dy = synth.dy_rows(w, rows) if backward else None
+        t0 = time.perf_counter()
+        if backward:
+            oracle.hyena_backward(v, xs, hs, dy, filter_row=fr, threads=n_threads)
+        else:
+            oracle.hyena_forward(v, xs, hs, filter_row=fr, threads=n_threads)
+        return time.perf_counter() - t0
+
+    # calibrate on one row, then size the sample for ~target core-seconds
+    per_row = max(run([0], 1), 1e-4)
     nrows = int(min(w.channels, max(threads, target_core_seconds / per_row)))
-    rows = list(range(nrows))
-    v, xs = synth.inputs(w, rows)
-    cs = sorted({r % w.D for r in rows})
-    hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
-                                   rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
-    hs = [hrows[n * len(cs):(n + 1) * len(cs)] for n in range(w.N)]
-    fr = [cs.index(r % w.D) for r in rows]
-    t0 = time.perf_counter()
-    oracle.hyena_forward(v, xs, hs, filter_row=fr, threads=threads)
-    dt = time.perf_counter() - t0
+    dt = run(list(range(nrows)), threads)
     value = nrows * w.L / dt / 1e9
-    sample = (f"{nrows} of {w.channels} (b,c) rows of {w.name}, all N={w.N} stages, "
-              f"{'direct O(L^2)' if w.L <= 8192 else 'radix-2 FFT'} causal conv, filters precomputed")
+    what = "backward (forward again, then gradients)" if backward else "forward"
+    sample = (f"{nrows} of {w.channels} (b,c) rows of {w.name}, {what}, all N={w.N} stages, "
+              f"{'direct O(L^2)' if w.L <= 8192 else 'radix-2 FFT'} causal sums, filters precomputed")
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
             "seconds": dt}
 
@@ -218,7 +254,10 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (default 1: B=4 D=768 L=2048 N=2 bf16)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward")
     args = ap.parse_args()
+    bwd = args.which == "backward"
+    metric = METRIC_BWD if bwd else METRIC
     if args.warmup < 3:
         args.warmup = 3
 
@@ -230,12 +269,12 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_sample(w)
-        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+        cb = oracle_sample(w, backward=bwd)
+        line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.channels * w.L / (cb["value"] * 1e9) * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N,
-                                                 "io": w.dtype},
+                                                 "io": w.dtype, "pass": args.which},
                 "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
                 "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -271,23 +310,32 @@ def main():
     base_x = [torch.from_numpy(x).view(w.B, w.D, w.L).to(dev).to(dt) for x in xs_np]
     base_h = [hy.filter_rfft(h[n]) for n in range(w.N)]
     del h
-    set_bytes = (w.N + 2) * w.channels * w.L * w.elem_bytes + sum(t.numel() for t in base_h)
+    base_dy = (torch.from_numpy(synth.dy_rows(wr)).view(w.B, w.D, w.L).to(dev).to(dt) if bwd else None)
+    set_bytes = ((w.N + 2 + (1 if bwd else 0)) * w.channels * w.L * w.elem_bytes
+                 + sum(t.numel() for t in base_h))
     nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    shared_out = None
+    if bwd:
+        # one set of outputs and one workspace, shared by every input set
+        first = hy.PreparedBackward(base_v, base_x, base_h, base_dy, stream=stream)
+        shared_out = (first.dv, first.dxs, first.dh, first._keep[4])
+
+    def prepared(v_s, x_s, h_s, dy_s, st):
+        if bwd:
+            dv_, dxs_, dh_, ws_ = shared_out
+            return hy.PreparedBackward(v_s, x_s, h_s, dy_s, dv=dv_, dxs=dxs_, dh=dh_, workspace=ws_, stream=st)
+        return hy.PreparedForward(v_s, x_s, h_s, stream=st)
+
     sets = []
     for s in range(nsets):
         if s == 0:
-            v_s, x_s, h_s = base_v, base_x, base_h
+            v_s, x_s, h_s, dy_s = base_v, base_x, base_h, base_dy
         else:
             v_s, x_s, h_s = base_v.clone(), [x.clone() for x in base_x], [t.clone() for t in base_h]
-        sets.append(hy.PreparedForward(v_s, x_s, h_s, stream=stream))
+            dy_s = base_dy.clone() if bwd else None
+        sets.append(prepared(v_s, x_s, h_s, dy_s, stream))
     torch.cuda.synchronize()
-    launches_per_step = 1 if w.L <= 8192 else None
-    if launches_per_step is None:
-        M, M1, MV = hy.spectrum_layout(w.L)
-        ws = hy.forward_workspace_bytes(w.B, w.D, w.L, w.N, dt == torch.bfloat16)
-        wave = ws // (8 * w.L)
-        waves = math.ceil(w.channels / wave)
-        launches_per_step = waves * (2 * w.N + 1)
+    launches_per_step = count_kernel_nodes(lambda st: prepared(base_v, base_x, base_h, base_dy, st))
 
     # warm-up
     for i in range(args.warmup):
@@ -321,25 +369,43 @@ def main():
     value = whole_job_throughput(K * w.channels * w.L, world, elapsed_ms)
     kernel_ms = statistics.mean(step_ms)
     peak, peak_kind = hbm_peak()
-    alg_bytes = w.roofline_bytes()
+    alg_bytes = backward_bytes(w) if bwd else w.roofline_bytes()
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs in, result out
     pin_v = base_v.cpu().pin_memory()
     pin_x = [x.cpu().pin_memory() for x in base_x]
-    pin_y = torch.empty_like(pin_v).pin_memory()
     dv = torch.empty_like(base_v)
     dxs = [torch.empty_like(x) for x in base_x]
-    e2e_fwd = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream)
-    h2d = (w.N + 1) * w.channels * w.L * w.elem_bytes
-    d2h = w.channels * w.L * w.elem_bytes
+    if bwd:
+        pin_dy = base_dy.cpu().pin_memory()
+        ddy = torch.empty_like(base_dy)
+        dv_s, dxs_s, dh_s, ws_s = shared_out
+        pin_out = [torch.empty_like(dv_s, device="cpu").pin_memory()] + \
+                  [torch.empty_like(t, device="cpu").pin_memory() for t in dxs_s] + \
+                  [torch.empty_like(dh_s, device="cpu").pin_memory()]
+        e2e_call = hy.PreparedBackward(dv, dxs, sets[0]._keep[2], ddy, dv=dv_s, dxs=dxs_s, dh=dh_s,
+                                       workspace=ws_s, stream=stream)
+        h2d = (w.N + 2) * w.channels * w.L * w.elem_bytes
+        d2h = (w.N + 1) * w.channels * w.L * w.elem_bytes + 4 * w.N * w.D * w.L
+    else:
+        pin_y = torch.empty_like(pin_v).pin_memory()
+        e2e_call = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream)
+        h2d = (w.N + 1) * w.channels * w.L * w.elem_bytes
+        d2h = w.channels * w.L * w.elem_bytes
 
     def e2e_step():
         dv.copy_(pin_v, non_blocking=True)
         for d, p in zip(dxs, pin_x):
             d.copy_(p, non_blocking=True)
-        y = e2e_fwd()
-        pin_y.copy_(y, non_blocking=True)
+        if bwd:
+            ddy.copy_(pin_dy, non_blocking=True)
+            gdv, gdxs, gdh = e2e_call()
+            for p, t in zip(pin_out, [gdv, *gdxs, gdh]):
+                p.copy_(t, non_blocking=True)
+        else:
+            y = e2e_call()
+            pin_y.copy_(y, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -360,17 +426,18 @@ def main():
     line = None
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
+            "metric": metric, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype,
+            "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype, "pass": args.which,
                        "global_batch": w.B * world, "parallelism": f"replicas x{world}",
                        "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
                              f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": measured_traffic(w.name),
+                         "frac": round(achieved / peak, 4),
+                         "traffic": None if bwd else measured_traffic(w.name),
                          "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
-                         "kernel": dominant_kernel(w)[0],
+                         "kernel": ("whole backward step (all its launches)" if bwd else dominant_kernel(w)[0]),
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
@@ -382,7 +449,7 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            cb = oracle_sample(w)
+            cb = oracle_sample(w, backward=bwd)
             line["cpu_baseline"] = {k: round(cb[k], 6) if k == "value" else cb[k]
                                     for k in ("value", "unit", "cores", "kind", "sample")}
         elif not args.no_cpu_baseline:

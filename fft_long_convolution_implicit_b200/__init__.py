@@ -337,3 +337,37 @@ class PreparedForward:
         if st != HYENA_OK:
             raise HyenaError(st, "hyena_forward")
         return self.y
+
+
+class PreparedBackward:
+    """hyena_backward with its arguments marshalled once (fixed tensors,
+    workspace and stream); calling it issues the C call only."""
+
+    def __init__(self, v, xs, hhats, dy, dv=None, dxs=None, dh=None, workspace=None, stream=None):
+        torch = _torch()
+        B, D, L = v.shape
+        N = len(xs)
+        code = _dtype_code(v)
+        self.dv = torch.empty_like(v) if dv is None else dv
+        self.dxs = [torch.empty_like(v) for _ in range(N)] if dxs is None else list(dxs)
+        self.dh = torch.empty((N, D, L), dtype=torch.float32, device=v.device) if dh is None else dh
+        need = backward_workspace_bytes(B, D, L, N, code == HYENA_BF16)
+        if need == 0:
+            _check(HYENA_ERR_INVALID_ARG, "hyena_backward_workspace_bytes")
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+        self._keep = (v, list(xs), list(hhats), dy, workspace)
+        self._x = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+        self._h = (ctypes.c_void_p * N)(*[_dev(h, "hhat").value for h in hhats])
+        self._dx = (ctypes.c_void_p * N)(*[_dev(t, "dx").value for t in self.dxs])
+        self._dh = (ctypes.c_void_p * N)(*[_dev(self.dh[n], "dh").value for n in range(N)])
+        self._args = (_dev(v, "v"), self._x, self._h, _dev(dy, "dy"), B, D, L, N, code, _dev(self.dv, "dv"),
+                      self._dx, self._dh, _dev(workspace, "workspace"),
+                      workspace.numel() * workspace.element_size(), _stream(stream))
+        self._fn = load().hyena_backward
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != HYENA_OK:
+            raise HyenaError(st, "hyena_backward")
+        return self.dv, self.dxs, self.dh
