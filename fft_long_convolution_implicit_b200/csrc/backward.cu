@@ -2,7 +2,7 @@
 // through the implicit-filter FFN.
 //
 // The pages print no backward formulas (they mention training at 1M tokens:
-// glossary "Hyena（ハイエナ）", section 応用); this is the chain rule through
+// glossary "Hyena（ハイエナ）", section 超長系列タスクでの優位性); this is the chain rule through
 // the forward definitions (order-N recurrence, "Hyena Hierarchy" digest,
 // 방법 / 프레임워크 개요; causal FIR sum, "02. 3つの Hyena 演算子", section 4):
 //   u_n = h_n * z_n,  z_{n+1} = x_n . u_n,  g_{N+1} = dy,  r_n = g_{n+1} . x_n

@@ -168,7 +168,7 @@ hyena_status hyena_forward_static_workspace(const void *v, const void *const *x,
 
 /*
  * Gradients (no counterpart printed on the pages, which only mention training
- * at 1M tokens: glossary "Hyena（ハイエナ）", section 応用). They are the chain
+ * at 1M tokens: glossary "Hyena（ハイエナ）", section 超長系列タスクでの優位性). They are the chain
  * rule through the definitions above:
  *   u_n = h_n * z_n,  z_{n+1} = x_n (.) u_n,  g_{N+1} = dy,  r_n = g_{n+1} (.) x_n
  *   dx_n       = g_{n+1} (.) u_n

@@ -326,7 +326,7 @@ int oracle_hyena_forward(const double *v, const double *x, const double *h,
 
 /*
  * The pages print no backward formulas (they mention training at 1M tokens:
- * glossary "Hyena（ハイエナ）", section "応用"). What follows is the chain
+ * glossary "Hyena（ハイエナ）", section "超長系列タスクでの優位性"). What follows is the chain
  * rule applied to the forward definitions above, nothing more:
  *   u_n = h_n conv z_n,  z_{n+1} = x_n * u_n,  y = z_{N+1}.
  * With g_{N+1} = dL/dy and r_n = g_{n+1} * x_n:
