@@ -276,20 +276,25 @@ static cudaError_t wave_lm(const FourStepLaunch& p, const Layout& y, cudaStream_
   return p.bf16 ? wave_t<LOGMV, MB, __nv_bfloat16>(p, y, s) : wave_t<LOGMV, MB, float>(p, y, s);
 }
 
-cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
-  if (y.logMV == 10 && y.mb == 1) return wave_lm<10, 1>(p, y, s);
-  if (y.logMV == 11 && y.mb == 1) return wave_lm<11, 1>(p, y, s);
-  if (y.logMV == 12) {
-    switch (y.mb) {
-      case 1: return wave_lm<12, 1>(p, y, s);
-      case 2: return wave_lm<12, 2>(p, y, s);
-      case 4: return wave_lm<12, 4>(p, y, s);
-      case 8: return wave_lm<12, 8>(p, y, s);
-      case 16: return wave_lm<12, 16>(p, y, s);
-      default: break;
-    }
+template <int LOGMV>
+static cudaError_t wave_l(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
+  switch (y.mb) {
+    case 1: return wave_lm<LOGMV, 1>(p, y, s);
+    case 2: return wave_lm<LOGMV, 2>(p, y, s);
+    case 4: return wave_lm<LOGMV, 4>(p, y, s);
+    case 8: return wave_lm<LOGMV, 8>(p, y, s);
+    case 16: return wave_lm<LOGMV, 16>(p, y, s);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaErrorInvalidValue;
+}
+
+// Row lengths make_layout produces: 1024 (L <= 2^18) and 4096 points.
+cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
+  switch (y.logMV) {
+    case 10: return wave_l<10>(p, y, s);
+    case 12: return wave_l<12>(p, y, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int LOGMV, int MB>
@@ -301,21 +306,26 @@ static cudaError_t spec_lm(const float* h, float2* spec, const float2* tables, i
   return launch_row<LOGMV, kPairSpectrum>(spec, spec, tables, y.M1, 1, 0, D, s);
 }
 
+template <int LOGMV>
+static cudaError_t spec_l(const float* h, float2* spec, const float2* tables, int D, const Layout& y,
+                          cudaStream_t s) {
+  switch (y.mb) {
+    case 1: return spec_lm<LOGMV, 1>(h, spec, tables, D, y, s);
+    case 2: return spec_lm<LOGMV, 2>(h, spec, tables, D, y, s);
+    case 4: return spec_lm<LOGMV, 4>(h, spec, tables, D, y, s);
+    case 8: return spec_lm<LOGMV, 8>(h, spec, tables, D, y, s);
+    case 16: return spec_lm<LOGMV, 16>(h, spec, tables, D, y, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D, const Layout& y,
                                      cudaStream_t s) {
-  if (y.logMV == 10 && y.mb == 1) return spec_lm<10, 1>(h, spec, tables, D, y, s);
-  if (y.logMV == 11 && y.mb == 1) return spec_lm<11, 1>(h, spec, tables, D, y, s);
-  if (y.logMV == 12) {
-    switch (y.mb) {
-      case 1: return spec_lm<12, 1>(h, spec, tables, D, y, s);
-      case 2: return spec_lm<12, 2>(h, spec, tables, D, y, s);
-      case 4: return spec_lm<12, 4>(h, spec, tables, D, y, s);
-      case 8: return spec_lm<12, 8>(h, spec, tables, D, y, s);
-      case 16: return spec_lm<12, 16>(h, spec, tables, D, y, s);
-      default: break;
-    }
+  switch (y.logMV) {
+    case 10: return spec_l<10>(h, spec, tables, D, y, s);
+    case 12: return spec_l<12>(h, spec, tables, D, y, s);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaErrorInvalidValue;
 }
 
 }  // namespace hyena

@@ -13,7 +13,9 @@ constexpr int kFusedMaxL = 8192;
 constexpr int kMinM = 128;          // smallest internal transform (zero-extended below)
 constexpr int kMaxL = 1 << 20;
 constexpr int kFourStepMaxMV = 4096;
+constexpr int kFourStepRowMV = 1024;   // preferred row length (measured fastest at L = 2^17)
 constexpr int kFourStepMinM1 = 16;
+constexpr int kFourStepMaxM1 = 256;    // columns: radix 16 x (M1 / 16) with M1 / 16 <= 16
 
 struct Layout {
   int L;        // caller's length
@@ -58,7 +60,10 @@ inline bool make_layout(int L, Layout* out) {
     y.mb = 0;
   } else {
     y.M = L;
-    y.M1 = L / kFourStepMaxMV;
+    // rows of 1024 points while the columns stay within 256 points; longer
+    // transforms use rows of 4096 points
+    y.M1 = L / kFourStepRowMV;
+    if (y.M1 > kFourStepMaxM1) y.M1 = L / kFourStepMaxMV;
     if (y.M1 < kFourStepMinM1) y.M1 = kFourStepMinM1;
     y.MV = L / y.M1;
     y.fourstep = true;

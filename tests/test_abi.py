@@ -49,7 +49,7 @@ def test_host_queries(lib):
     M, M1, MV = hy.spectrum_layout(1 << 20)
     assert M == 1 << 20 and M1 * MV == M and MV <= 4096
     M, M1, MV = hy.spectrum_layout(131072)
-    assert (M1, MV) == (32, 4096)
+    assert (M1, MV) == (128, 1024)
     assert hy.forward_workspace_bytes(4, 768, 2048, 2, True) == 0
     ws = hy.forward_workspace_bytes(1, 256, 131072, 2, True)
     assert ws % (131072 * 8) == 0 and ws >= 131072 * 8
