@@ -55,13 +55,22 @@ KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "tc": ("tc_fused.cu", "fft_engine.cuh", "layout.h"),
+    "tc05": ("tc05.cu", "fft_engine.cuh", "kernels.cuh", "layout.h"),
 }
+
+
+def tc05_built() -> bool:
+    """True when the library was built with the tcgen05 forward (build.py --tc05)."""
+    from fft_long_convolution_implicit_b200 import build as hybuild
+    return hybuild.built_tc05()
 
 
 def dominant_kernel(w: synth.Workload) -> tuple[str, str]:
     """(kernel name, source set) of the launch that dominates one forward."""
     if w.L > 8192:
         return "four-step column/row kernels (whole step)", "fourstep"
+    if w.dtype == "bf16" and w.B % 2 == 0 and w.L == 2048 and tc05_built():
+        return "tc05_forward_kernel", "tc05"
     if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
         return "tc_forward_kernel", "tc"
     return "fused_forward_kernel", "fused"

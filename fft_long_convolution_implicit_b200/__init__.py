@@ -20,7 +20,7 @@ import os
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "lib", "libhyena_b200.so")
 
-HYENA_OK, HYENA_ERR_INVALID_ARG, HYENA_ERR_UNSUPPORTED, HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA = range(5)
+HYENA_OK, HYENA_ERR_INVALID_ARG, HYENA_ERR_UNSUPPORTED, HYENA_ERR_WORKSPACE, HYENA_ERR_CUDA, HYENA_ERR_TIMEOUT = range(6)
 HYENA_F32, HYENA_BF16 = 0, 1
 
 # exported symbols (kept in step with include/hyena.h)
@@ -28,7 +28,7 @@ EXPORTS = (
     "hyena_filter_generate", "hyena_filter_spectrum_bytes", "hyena_filter_rfft", "hyena_spectrum_layout",
     "hyena_forward_workspace_bytes", "hyena_forward", "hyena_status_string", "hyena_last_cuda_error",
     "hyena_abi_version", "hyena_forward_static_workspace", "hyena_backward_workspace_bytes", "hyena_backward",
-    "hyena_filter_backward_workspace_bytes", "hyena_filter_backward",
+    "hyena_filter_backward_workspace_bytes", "hyena_filter_backward", "hyena_device_timeouts",
 )
 
 
@@ -93,6 +93,8 @@ def load() -> ctypes.CDLL:
     l.hyena_status_string.restype = ctypes.c_char_p
     l.hyena_last_cuda_error.argtypes = []
     l.hyena_last_cuda_error.restype = ctypes.c_char_p
+    l.hyena_device_timeouts.argtypes = []
+    l.hyena_device_timeouts.restype = i
     l.hyena_abi_version.argtypes = []
     l.hyena_abi_version.restype = i
     _lib = l
@@ -134,6 +136,12 @@ def _dev(t, name):
 
 def abi_version() -> int:
     return load().hyena_abi_version()
+
+
+def check_device_timeouts():
+    """Raise HyenaError(HYENA_ERR_TIMEOUT) if a bounded device wait ran out
+    since the last check (synchronises with the device; clears the flag)."""
+    _check(load().hyena_device_timeouts(), "hyena_device_timeouts")
 
 
 def filter_spectrum_bytes(D: int, L: int) -> int:

@@ -21,6 +21,13 @@ hyena_status cuda_fail(cudaError_t e) {
 
 bool aligned16(const void* p) { return p && ((reinterpret_cast<uintptr_t>(p) & 15u) == 0); }
 
+// L = 2048 bf16 pairs: tcgen05 kernel (tc05.cu) when built with HYENA_TC05=1,
+// otherwise the mma.sync kernel (tc_fused.cu)
+#ifndef HYENA_TC05
+#define HYENA_TC05 0
+#endif
+constexpr bool kUseTc05 = HYENA_TC05 != 0;
+
 // L2-sized wave of four-step channels
 constexpr size_t kWaveTargetBytes = size_t(48) << 20;
 constexpr long long kMaxGridY = 65535;
@@ -95,7 +102,7 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
       // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
       for (int n = 0; n < N; ++n)
         p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
-      e = launch_tc_forward(p, ly, s);
+      e = (kUseTc05 && ly.R0 == 16) ? launch_tc05_forward(p, s) : launch_tc_forward(p, ly, s);
     } else {
       e = launch_fused_forward(p, ly.logMV, s);
     }
@@ -143,7 +150,8 @@ cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, con
   if (!ly.fourstep) {
     e = launch_fused_spectrum(h, spec, tables, rows, ly.L, ly.logMV, s);
     if (e == cudaSuccess && with_tc && ly.tc)
-      e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
+      e = (kUseTc05 && ly.R0 == 16) ? launch_tc05_spectrum(spec, spec + tc_spectrum_offset(ly, rows), rows, ly.M, s)
+                                    : launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
   } else {
     for (long long c0 = 0; c0 < rows && e == cudaSuccess; c0 += kMaxGridY) {
       const int nd = (int)((rows - c0) < kMaxGridY ? (rows - c0) : kMaxGridY);
@@ -164,11 +172,18 @@ const char* hyena_status_string(hyena_status s) {
     case HYENA_ERR_UNSUPPORTED: return "unsupported length (L must be a power of two in [16, 2^20])";
     case HYENA_ERR_WORKSPACE: return "workspace missing or too small";
     case HYENA_ERR_CUDA: return "CUDA error";
+    case HYENA_ERR_TIMEOUT: return "a bounded device wait ran out (results of the affected call are invalid)";
   }
   return "unknown status";
 }
 
 const char* hyena_last_cuda_error(void) { return g_last_cuda_error; }
+
+hyena_status hyena_device_timeouts(void) {
+  const int v = tc05_read_and_clear_timeout();
+  if (v < 0) return cuda_fail(cudaGetLastError());
+  return v ? HYENA_ERR_TIMEOUT : HYENA_OK;
+}
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {
   Layout y;

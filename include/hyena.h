@@ -48,7 +48,8 @@ typedef enum {
   HYENA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad count or dtype */
   HYENA_ERR_UNSUPPORTED = 2,   /* L not a power of two in [16, 2^20] */
   HYENA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
-  HYENA_ERR_CUDA = 4           /* a CUDA launch or attribute call failed */
+  HYENA_ERR_CUDA = 4,          /* a CUDA launch or attribute call failed */
+  HYENA_ERR_TIMEOUT = 5        /* a bounded device-side wait ran out (see hyena_device_timeouts) */
 } hyena_status;
 
 typedef enum { HYENA_F32 = 0, HYENA_BF16 = 1 } hyena_dtype;
@@ -229,6 +230,18 @@ const char *hyena_status_string(hyena_status s);
 
 /* Text of the last CUDA error seen by this thread inside the library ("" if none). */
 const char *hyena_last_cuda_error(void);
+
+/*
+ * Kernels that wait on mbarriers for asynchronous tensor-core work (the
+ * tcgen05 forward for bf16, L = 2048, B even, in libraries built with
+ * HYENA_TC05) bound every wait by an iteration limit; a wait that runs out
+ * makes every thread block of that launch stop early (its outputs are then
+ * invalid) and sets a sticky flag on the current device. This call
+ * synchronises with the device, reads and clears the flag: HYENA_OK if no
+ * wait ran out since the last call, HYENA_ERR_TIMEOUT otherwise
+ * (HYENA_ERR_CUDA if it cannot be read).
+ */
+hyena_status hyena_device_timeouts(void);
 
 /* HYENA_ABI_VERSION of the loaded library. */
 int hyena_abi_version(void);

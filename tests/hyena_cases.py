@@ -42,6 +42,7 @@ def gpu_run(w: synth.Workload, v=None, xs=None, keep_h: bool = False):
     txs = [upload(x, w) for x in xs]
     y = hy.forward(tv, txs, hh)
     torch.cuda.synchronize()
+    hy.check_device_timeouts()
     y_np = y.float().cpu().numpy().reshape(w.channels, w.L)
     h_np = h.cpu().numpy() if keep_h else None
     return y_np, h_np, (v, xs, wt)
