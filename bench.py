@@ -264,13 +264,19 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward")
+    ap.add_argument("--shape", default=None,
+                    help="N,dtype,B,D,L: a custom shape instead of --config (small ncu captures)")
     args = ap.parse_args()
     bwd = args.which == "backward"
     metric = METRIC_BWD if bwd else METRIC
     if args.warmup < 3:
         args.warmup = 3
 
-    w = synth.workload(args.config)
+    if args.shape:
+        n_, dt_, b_, d_, l_ = args.shape.split(",")
+        w = synth.custom(int(n_), dt_, int(b_), int(d_), int(l_))
+    else:
+        w = synth.workload(args.config)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
