@@ -65,6 +65,8 @@ def lib():
         l.oracle_hyena_backward.restype = i32
         l.oracle_filter_backward.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, d, d, P,
                                              P, P, P, P, P, P, i32]
+        l.oracle_striped_forward.argtypes = [P, P, P, P, P, P, i32, P, i32, P, i64, i64, P, i32]
+        l.oracle_striped_forward.restype = i32
         _lib = l
     return _lib
 
@@ -233,3 +235,21 @@ def filter_backward(weights: dict, N: int, D: int, L: int, alpha_lo: float, alph
                                  *(_p(out[k]) for k in ("W1", "b1", "W2", "b2", "W3", "b3")),
                                  threads or default_threads())
     return out
+
+
+def striped_forward(xq, xk, xv, hT, hH, hK, hG, filter_row=None, threads: int | None = None) -> np.ndarray:
+    """StripedHyena-form operator y = (hT*xq) . (hG * ((hH*xk) . (hK*xv))) with
+    causal FIR sums. x*: [C][L]; hT, hH, hK: [F][lf]; hG: [F][lg]."""
+    xq, xk, xv = (_f64(np.atleast_2d(a)) for a in (xq, xk, xv))
+    C, L = xq.shape
+    hT, hH, hK, hG = (_f64(np.atleast_2d(a)) for a in (hT, hH, hK, hG))
+    F, lf = hT.shape
+    lg = hG.shape[1]
+    assert hH.shape == hK.shape == (F, lf) and hG.shape[0] == F
+    fr = np.ascontiguousarray(np.arange(C) if filter_row is None else filter_row, dtype=np.int32)
+    y = np.empty((C, L))
+    rc = lib().oracle_striped_forward(_p(xq), _p(xk), _p(xv), _p(hT), _p(hH), _p(hK), lf, _p(hG), lg,
+                                      _p(fr), C, L, _p(y), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle_striped_forward rejected its arguments")
+    return y

@@ -598,3 +598,86 @@ void oracle_filter_backward(const float *W1, const float *b1, const float *W2, c
     }
     free(part); free(th); free(jobs);
 }
+
+/* ------------------------------------------------------------------------ */
+/* StripedHyena-form operator                                               */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * "02. 3つの Hyena 演算子", section 2 (the operator structure) and section 4
+ * (the FIR sum y_t = sum_{k < l_h} h_k x_{t-k}):
+ *   q = h_T * xq,  k = h_H * xk,  v = h_K * xv      (short explicit FIRs)
+ *   y = q (.) (h_G * (k (.) v))
+ * (the dense projections W, U, P, M of that section are outside this
+ * operator: xq, xk, xv are their outputs). Every * is the causal FIR sum,
+ * zero before t = 0. One channel, length L; filters of length lf (featurizers)
+ * and lg (inner).
+ */
+static void fir_causal(const double *h, int lh, const double *x, int64_t L, double *out)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        double acc = 0.0;
+        for (int j = 0; j < lh && j <= t; ++j) acc += h[j] * x[t - j];
+        out[t] = acc;
+    }
+}
+
+void oracle_striped_channel(const double *xq, const double *xk, const double *xv,
+                            const double *hT, const double *hH, const double *hK, int lf,
+                            const double *hG, int lg, int64_t L, double *y)
+{
+    double *q = (double *)malloc(sizeof(double) * L), *k = (double *)malloc(sizeof(double) * L);
+    double *v = (double *)malloc(sizeof(double) * L), *w = (double *)malloc(sizeof(double) * L);
+    fir_causal(hT, lf, xq, L, q);
+    fir_causal(hH, lf, xk, L, k);
+    fir_causal(hK, lf, xv, L, v);
+    for (int64_t t = 0; t < L; ++t) k[t] *= v[t];
+    fir_causal(hG, lg, k, L, w);
+    for (int64_t t = 0; t < L; ++t) y[t] = q[t] * w[t];
+    free(q); free(k); free(v); free(w);
+}
+
+typedef struct {
+    const double *xq, *xk, *xv, *hT, *hH, *hK, *hG;
+    const int *filter_row;
+    int lf, lg;
+    int64_t L;
+    double *y;
+    int begin, end;
+} striped_job;
+
+static void *striped_worker(void *arg)
+{
+    striped_job *j = (striped_job *)arg;
+    for (int r = j->begin; r < j->end; ++r) {
+        const int f = j->filter_row[r];
+        const size_t o = (size_t)r * j->L;
+        oracle_striped_channel(j->xq + o, j->xk + o, j->xv + o, j->hT + (size_t)f * j->lf,
+                               j->hH + (size_t)f * j->lf, j->hK + (size_t)f * j->lf, j->lf,
+                               j->hG + (size_t)f * j->lg, j->lg, j->L, j->y + o);
+    }
+    return NULL;
+}
+
+/* C channels [C][L]; filters [F][lf] / [F][lg], channel r uses row filter_row[r]. */
+int oracle_striped_forward(const double *xq, const double *xk, const double *xv,
+                           const double *hT, const double *hH, const double *hK, int lf,
+                           const double *hG, int lg, const int *filter_row, int64_t C, int64_t L,
+                           double *y, int n_threads)
+{
+    if (lf < 1 || lg < 1 || L < 1 || C < 0) return 1;
+    if (C == 0) return 0;
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > C) n_threads = (int)C;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n_threads);
+    striped_job *jobs = (striped_job *)malloc(sizeof(striped_job) * n_threads);
+    for (int i = 0; i < n_threads; ++i) {
+        striped_job j = {xq, xk, xv, hT, hH, hK, hG, filter_row, lf, lg, L, y,
+                         (int)(C * i / n_threads), (int)(C * (i + 1) / n_threads)};
+        jobs[i] = j;
+        pthread_create(&th[i], NULL, striped_worker, &jobs[i]);
+    }
+    for (int i = 0; i < n_threads; ++i) pthread_join(th[i], NULL);
+    free(th); free(jobs);
+    return 0;
+}
