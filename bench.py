@@ -19,6 +19,9 @@ same workload (rank 0 only).
 gradient dy), same workload and conventions; its roofline counts the bytes
 the gradients must move at least: v, x_n, dy and the spectra in, dv, dx_n
 and dh_n out.
+--pass striped times the StripedHyena-form operator q . (hG * (k . v)) with
+Hyena-SE filters (featurizers of 4 taps, inner filter of 7) on the workload's
+B, D, L: three inputs and one output of B*D*L elements each.
 """
 from __future__ import annotations
 
@@ -42,6 +45,8 @@ import synth  # noqa: E402
 
 METRIC = "Hyena order-N fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
 METRIC_BWD = "Hyena order-N bwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
+METRIC_STRIPED = "StripedHyena-SE fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
+STRIPED_LF, STRIPED_LG = 4, 7
 UNIT = "1e9 B*D*L/s"
 KERNEL_SOURCES = os.path.join(ROOT, "fft_long_convolution_implicit_b200", "csrc")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
@@ -252,6 +257,26 @@ def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0, backward
             "seconds": dt}
 
 
+def oracle_striped_sample(w: synth.Workload, target_core_seconds: float = 8.0):
+    """The float64 StripedHyena-form oracle on a bounded sample of rows."""
+    import oracle
+    threads = host_cores()
+    hT, hH, hK, hG = synth.striped_filters(w, STRIPED_LF, STRIPED_LG)
+
+    def run(rows, n_threads):
+        xv, (xq, xk) = synth.inputs(synth.Workload(**{**w.__dict__, "N": 2}), rows)
+        t0 = time.perf_counter()
+        oracle.striped_forward(xq, xk, xv, hT, hH, hK, hG, filter_row=[r % w.D for r in rows], threads=n_threads)
+        return time.perf_counter() - t0
+
+    per_row = max(run([0], 1), 1e-5)
+    nrows = int(min(w.channels, max(threads, target_core_seconds / per_row)))
+    dt = run(list(range(nrows)), threads)
+    return {"value": nrows * w.L / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{nrows} of {w.channels} (b,c) rows, StripedHyena-SE (lf={STRIPED_LF}, lg={STRIPED_LG}), "
+                      f"direct FIR sums", "seconds": dt}
+
+
 # ---------------------------------------------------------------- main --
 
 def main():
@@ -263,12 +288,13 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (default 1: B=4 D=768 L=2048 N=2 bf16)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", choices=["forward", "backward"], default="forward")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward", "striped"], default="forward")
     ap.add_argument("--shape", default=None,
                     help="N,dtype,B,D,L: a custom shape instead of --config (small ncu captures)")
     args = ap.parse_args()
     bwd = args.which == "backward"
-    metric = METRIC_BWD if bwd else METRIC
+    striped = args.which == "striped"
+    metric = METRIC_BWD if bwd else (METRIC_STRIPED if striped else METRIC)
     if args.warmup < 3:
         args.warmup = 3
 
@@ -284,7 +310,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_sample(w, backward=bwd)
+        cb = oracle_striped_sample(w) if striped else oracle_sample(w, backward=bwd)
         line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.channels * w.L / (cb["value"] * 1e9) * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -317,6 +343,8 @@ def main():
 
     # inputs of this rank (seeded per rank), weights and cached spectra
     wr = rank_workload(w, rank)
+    if striped and w.N < 2:
+        wr = synth.Workload(**{**wr.__dict__, "N": 2})
     v_np, xs_np = synth.inputs(wr)
     wt = synth.filter_weights(wr)
     tw = {k: torch.from_numpy(np.ascontiguousarray(a)).to(dev) for k, a in wt.items()}
@@ -328,6 +356,8 @@ def main():
     base_dy = (torch.from_numpy(synth.dy_rows(wr)).view(w.B, w.D, w.L).to(dev).to(dt) if bwd else None)
     set_bytes = ((w.N + 2 + (1 if bwd else 0)) * w.channels * w.L * w.elem_bytes
                  + sum(t.numel() for t in base_h))
+    if striped:
+        set_bytes = 3 * w.channels * w.L * w.elem_bytes
     nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
     shared_out = None
     if bwd:
@@ -335,7 +365,13 @@ def main():
         first = hy.PreparedBackward(base_v, base_x, base_h, base_dy, stream=stream)
         shared_out = (first.dv, first.dxs, first.dh, first._keep[4])
 
+    if striped:
+        sf = [torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+              for a in synth.striped_filters(wr, STRIPED_LF, STRIPED_LG)]
+
     def prepared(v_s, x_s, h_s, dy_s, st):
+        if striped:
+            return hy.PreparedStriped(x_s[0], x_s[1], v_s, *sf, stream=st)
         if bwd:
             dv_, dxs_, dh_, ws_ = shared_out
             return hy.PreparedBackward(v_s, x_s, h_s, dy_s, dv=dv_, dxs=dxs_, dh=dh_, workspace=ws_, stream=st)
@@ -384,7 +420,12 @@ def main():
     value = whole_job_throughput(K * w.channels * w.L, world, elapsed_ms)
     kernel_ms = statistics.mean(step_ms)
     peak, peak_kind = hbm_peak()
-    alg_bytes = backward_bytes(w) if bwd else w.roofline_bytes()
+    if bwd:
+        alg_bytes = backward_bytes(w)
+    elif striped:
+        alg_bytes = 4 * w.channels * w.L * w.elem_bytes + 4 * w.D * (3 * STRIPED_LF + STRIPED_LG)
+    else:
+        alg_bytes = w.roofline_bytes()
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs in, result out
@@ -403,6 +444,11 @@ def main():
                                        workspace=ws_s, stream=stream)
         h2d = (w.N + 2) * w.channels * w.L * w.elem_bytes
         d2h = (w.N + 1) * w.channels * w.L * w.elem_bytes + 4 * w.N * w.D * w.L
+    elif striped:
+        pin_y = torch.empty_like(pin_v).pin_memory()
+        e2e_call = hy.PreparedStriped(dxs[0], dxs[1], dv, *sf, stream=stream)
+        h2d = 3 * w.channels * w.L * w.elem_bytes
+        d2h = w.channels * w.L * w.elem_bytes
     else:
         pin_y = torch.empty_like(pin_v).pin_memory()
         e2e_call = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream)
@@ -450,9 +496,10 @@ def main():
                              f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": None if bwd else measured_traffic(w.name),
+                         "traffic": None if (bwd or striped) else measured_traffic(w.name),
                          "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
-                         "kernel": ("whole backward step (all its launches)" if bwd else dominant_kernel(w)[0]),
+                         "kernel": ("whole backward step (all its launches)" if bwd else
+                                    ("striped_kernel (fused FIR)" if striped else dominant_kernel(w)[0])),
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
@@ -464,7 +511,7 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         if not args.no_cpu_baseline and world == 1:
-            cb = oracle_sample(w, backward=bwd)
+            cb = oracle_striped_sample(w) if striped else oracle_sample(w, backward=bwd)
             line["cpu_baseline"] = {k: round(cb[k], 6) if k == "value" else cb[k]
                                     for k in ("value", "unit", "cores", "kind", "sample")}
         elif not args.no_cpu_baseline:

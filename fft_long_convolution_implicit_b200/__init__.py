@@ -29,6 +29,7 @@ EXPORTS = (
     "hyena_forward_workspace_bytes", "hyena_forward", "hyena_status_string", "hyena_last_cuda_error",
     "hyena_abi_version", "hyena_forward_static_workspace", "hyena_backward_workspace_bytes", "hyena_backward",
     "hyena_filter_backward_workspace_bytes", "hyena_filter_backward", "hyena_device_timeouts",
+    "hyena_striped_forward", "hyena_striped_featurize", "hyena_filter_exponential",
 )
 
 
@@ -93,6 +94,12 @@ def load() -> ctypes.CDLL:
     l.hyena_status_string.restype = ctypes.c_char_p
     l.hyena_last_cuda_error.argtypes = []
     l.hyena_last_cuda_error.restype = ctypes.c_char_p
+    l.hyena_striped_forward.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i, i, P, P]
+    l.hyena_striped_forward.restype = i
+    l.hyena_striped_featurize.argtypes = [P, P, P, P, P, P, i, i, i, i, i, P, P, P]
+    l.hyena_striped_featurize.restype = i
+    l.hyena_filter_exponential.argtypes = [P, P, i, i, i, P, P]
+    l.hyena_filter_exponential.restype = i
     l.hyena_device_timeouts.argtypes = []
     l.hyena_device_timeouts.restype = i
     l.hyena_abi_version.argtypes = []
@@ -379,3 +386,66 @@ class PreparedBackward:
         if st != HYENA_OK:
             raise HyenaError(st, "hyena_backward")
         return self.dv, self.dxs, self.dh
+
+
+def striped_forward(xq, xk, xv, hT, hH, hK, hG, y=None, stream=None):
+    """StripedHyena-form operator y = (hT*xq) . (hG * ((hH*xk) . (hK*xv))) with
+    causal FIR sums (SE / MR inner filters). x*: [B][D][L] float32 or bfloat16;
+    hT, hH, hK: float32 [D][lf]; hG: float32 [D][lg]."""
+    torch = _torch()
+    B, D, L = xq.shape
+    code = _dtype_code(xq)
+    for t in (xk, xv):
+        if t.shape != xq.shape or t.dtype != xq.dtype:
+            raise ValueError("xq, xk, xv must match in shape and dtype")
+    lf, lg = hT.shape[1], hG.shape[1]
+    y = torch.empty_like(xq) if y is None else y
+    _check(load().hyena_striped_forward(_dev(xq, "xq"), _dev(xk, "xk"), _dev(xv, "xv"), _dev(hT, "hT"),
+                                        _dev(hH, "hH"), _dev(hK, "hK"), lf, _dev(hG, "hG"), lg, B, D, L, code,
+                                        _dev(y, "y"), _stream(stream)), "hyena_striped_forward")
+    return y
+
+
+def striped_featurize(xq, xk, xv, hT, hH, hK, q=None, u=None, stream=None):
+    """(q, u) = (hT*xq, (hH*xk) . (hK*xv)) for the long-filter (LI) form:
+    y = forward(u, [q], [filter_rfft(hG)])."""
+    torch = _torch()
+    B, D, L = xq.shape
+    code = _dtype_code(xq)
+    lf = hT.shape[1]
+    q = torch.empty_like(xq) if q is None else q
+    u = torch.empty_like(xq) if u is None else u
+    _check(load().hyena_striped_featurize(_dev(xq, "xq"), _dev(xk, "xk"), _dev(xv, "xv"), _dev(hT, "hT"),
+                                          _dev(hH, "hH"), _dev(hK, "hK"), lf, B, D, L, code, _dev(q, "q"),
+                                          _dev(u, "u"), _stream(stream)), "hyena_striped_featurize")
+    return q, u
+
+
+def filter_exponential(R, lam, L: int, h=None, stream=None):
+    """Hyena-LI filter h[c][t] = sum_n R[c][n] lam[c][n]^t, float32 [D][L]."""
+    torch = _torch()
+    D, d = R.shape
+    h = torch.empty((D, L), dtype=torch.float32, device=R.device) if h is None else h
+    _check(load().hyena_filter_exponential(_dev(R, "R"), _dev(lam, "lambda"), d, D, L, _dev(h, "h"),
+                                           _stream(stream)), "hyena_filter_exponential")
+    return h
+
+
+class PreparedStriped:
+    """hyena_striped_forward with its arguments marshalled once."""
+
+    def __init__(self, xq, xk, xv, hT, hH, hK, hG, y=None, stream=None):
+        torch = _torch()
+        B, D, L = xq.shape
+        self.y = torch.empty_like(xq) if y is None else y
+        self._keep = (xq, xk, xv, hT, hH, hK, hG)
+        self._args = (_dev(xq, "xq"), _dev(xk, "xk"), _dev(xv, "xv"), _dev(hT, "hT"), _dev(hH, "hH"),
+                      _dev(hK, "hK"), hT.shape[1], _dev(hG, "hG"), hG.shape[1], B, D, L, _dtype_code(xq),
+                      _dev(self.y, "y"), _stream(stream))
+        self._fn = load().hyena_striped_forward
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != HYENA_OK:
+            raise HyenaError(st, "hyena_striped_forward")
+        return self.y

@@ -87,6 +87,14 @@ cudaError_t launch_tc_spectrum(const float2* nat, float2* tcs, float2* tables, i
 cudaError_t launch_tc05_forward(const FusedLaunch& p, cudaStream_t s);
 cudaError_t launch_tc05_spectrum(const float2* nat, float2* tcs, int D, int M, cudaStream_t s);
 int tc05_read_and_clear_timeout();
+// StripedHyena-form operator: featurizer length <= kMaxStripedLF, explicit
+// inner filter length <= kMaxStripedLG. hG == nullptr: featurize only (q, u).
+constexpr int kMaxStripedLF = 16;
+constexpr int kMaxStripedLG = 1024;
+cudaError_t launch_striped(const void* xq, const void* xk, const void* xv, const float* hT, const float* hH,
+                           const float* hK, int lf, const float* hG, int lg, int B, int D, int L, bool bf16, void* y,
+                           void* q, void* u, cudaStream_t s);
+cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D, int L, float* h, cudaStream_t s);
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
                                      const Layout& y, cudaStream_t s);

@@ -232,6 +232,43 @@ const char *hyena_status_string(hyena_status s);
 const char *hyena_last_cuda_error(void);
 
 /*
+ * StripedHyena-form operator ("02. 3つの Hyena 演算子", section 2, the operator
+ * structure; section 3, the SE / MR / LI variants; section 4, the FIR sum
+ * y_t = sum_{k < l_h} h_k x_{t-k}):
+ *   q = hT * xq,  k = hH * xk,  v = hK * xv     (short explicit featurizers)
+ *   y = q (.) (hG * (k (.) v))
+ * where * is the causal FIR sum (zero before t = 0). xq, xk, xv are the
+ * outputs of the operator's dense input projections (not part of this call).
+ *   xq, xk, xv, y: device [B][D][L] dtype, y not aliasing an input
+ *   hT, hH, hK:    device float32 [D][lf], 1 <= lf <= 16
+ *   hG:            device float32 [D][lg], 1 <= lg <= 1024 (SE: a few taps;
+ *                  MR: hundreds, e.g. an explicit filter times a decay)
+ * Any L >= 1. Arithmetic in float32; bf16 results rounded to nearest even.
+ */
+hyena_status hyena_striped_forward(const void *xq, const void *xk, const void *xv, const float *hT, const float *hH,
+                                   const float *hK, int lf, const float *hG, int lg, int B, int D, int L,
+                                   hyena_dtype dtype, void *y, hyena_stream stream);
+
+/*
+ * The featurizer half of the operator for a long implicit inner filter
+ * (Hyena-LI): q = hT * xq and u = (hH * xk) (.) (hK * xv), device [B][D][L]
+ * dtype. The operator is then y = hyena_forward(u, {q}, {hyena_filter_rfft(hG)},
+ * N = 1). Arguments as in hyena_striped_forward.
+ */
+hyena_status hyena_striped_featurize(const void *xq, const void *xk, const void *xv, const float *hT,
+                                     const float *hH, const float *hK, int lf, int B, int D, int L,
+                                     hyena_dtype dtype, void *q, void *u, hyena_stream stream);
+
+/*
+ * Hyena-LI filter ("02. 3つの Hyena 演算子", section 3): a sum of real
+ * exponentials, h[c][t] = sum_{n < d} R[c][n] lambda[c][n]^t for t < L (the
+ * page's exponent t - 1 with 1-based t). R, lambda: device float32 [D][d],
+ * 1 <= d <= 64; h: device float32 [D][L].
+ */
+hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d, int D, int L, float *h,
+                                      hyena_stream stream);
+
+/*
  * Kernels that wait on mbarriers for asynchronous tensor-core work (the
  * tcgen05 forward for bf16, L = 2048, B even, in libraries built with
  * HYENA_TC05) bound every wait by an iteration limit; a wait that runs out

@@ -253,3 +253,12 @@ def striped_forward(xq, xk, xv, hT, hH, hK, hG, filter_row=None, threads: int | 
     if rc != 0:
         raise ValueError("oracle_striped_forward rejected its arguments")
     return y
+
+
+def exponential_filter(R, lam, L: int) -> np.ndarray:
+    """Hyena-LI filter ("02. 3つの Hyena 演算子", section 3): h[c][t] =
+    sum_n R[c][n] lam[c][n]^t for t < L (0-based lag t; the page writes
+    lambda^(t-1) with 1-based t). float64, evaluated term by term."""
+    R, lam = _f64(np.atleast_2d(R)), _f64(np.atleast_2d(lam))
+    t = np.arange(L, dtype=np.float64)
+    return np.einsum("cn,cnt->ct", R, lam[:, :, None] ** t[None, None, :])

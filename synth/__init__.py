@@ -19,7 +19,8 @@ tensor can be regenerated on its own:
 Tensor ids: 0 = v, n = x_n (n = 1..N), 101..106 = W1, b1, W2, b2, W3, b3,
 200 = the 4 x D embedding table E, 201 = the symbol stream, 300 = the loss
 gradient dy fed to the backward, 301 = a filter gradient dh fed to the
-filter-weight backward on its own.
+filter-weight backward on its own, 400..403 = the StripedHyena-form filters
+hT, hH, hK, hG, 404/405 = the Hyena-LI exponential weights R and rates lambda.
 """
 from __future__ import annotations
 
@@ -242,6 +243,26 @@ def dy_rows(w: Workload, rows: list[int] | None = None) -> np.ndarray:
 def dh_rows(w: Workload) -> np.ndarray:
     """A filter gradient dL/dh, float32 [N][D][L] of N(0,1) values."""
     return normal(w.seed, TID_DH, 0, w.N * w.D * w.L).astype(np.float32).reshape(w.N, w.D, w.L)
+
+
+def striped_filters(w: Workload, lf: int, lg: int):
+    """Featurizers hT, hH, hK: float32 [D][lf] of N(0,1)/sqrt(lf); inner hG:
+    float32 [D][lg] of N(0,1)/sqrt(lg) times exp(-4 t / lg) (an MR-style decay)."""
+    def nrm(tid, cols, scale):
+        return (normal(w.seed, tid, 0, w.D * cols).reshape(w.D, cols) * scale).astype(np.float32)
+    hT, hH, hK = (nrm(400 + i, lf, 1 / math.sqrt(lf)) for i in range(3))
+    decay = np.exp(-4.0 * np.arange(lg) / lg)
+    hG = (nrm(403, lg, 1 / math.sqrt(lg)) * decay).astype(np.float32)
+    return hT, hH, hK, hG
+
+
+def exponential_params(w: Workload, d: int):
+    """Hyena-LI weights: R [D][d] of N(0,1)/sqrt(d), rates lambda [D][d]
+    uniform in (0.5, 1 - 2/L) (decaying within the sequence)."""
+    R = (normal(w.seed, 404, 0, w.D * d).reshape(w.D, d) / math.sqrt(d)).astype(np.float32)
+    u = uniform(w.seed, 405, 0, w.D * d).reshape(w.D, d)
+    lam = (0.5 + (0.5 - 2.0 / max(w.L, 4)) * u).astype(np.float32)
+    return R, lam
 
 
 def sample_rows(w: Workload, count: int, salt: int = 0) -> list[int]:

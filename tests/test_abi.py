@@ -123,3 +123,19 @@ def test_backward_queries_and_host_rejections(lib):
     assert fb(None, 2, 4, 256, 0.5, 20.0, p, ctypes.byref(g), p, need, None) == hy.HYENA_ERR_INVALID_ARG
     bad = hy.FilterGrads(16, 16, 16, 16, None, 16)
     assert fb(ctypes.byref(fp), 2, 4, 256, 0.5, 20.0, p, ctypes.byref(bad), p, need, None) == hy.HYENA_ERR_INVALID_ARG
+
+
+def test_striped_host_rejections(lib):
+    p = ctypes.c_void_p(16)
+    f = lib.hyena_striped_forward
+    ok = (p, p, p, p, p, p, 4, p, 7, 2, 3, 100, hy.HYENA_BF16, p, None)
+    bad_lf = (p, p, p, p, p, p, 17, p, 7, 2, 3, 100, hy.HYENA_BF16, p, None)
+    bad_lg = (p, p, p, p, p, p, 4, p, 1025, 2, 3, 100, hy.HYENA_BF16, p, None)
+    bad_L = (p, p, p, p, p, p, 4, p, 7, 2, 3, 0, hy.HYENA_BF16, p, None)
+    mis = (ctypes.c_void_p(24), p, p, p, p, p, 4, p, 7, 2, 3, 100, hy.HYENA_BF16, p, None)
+    for args in (bad_lf, bad_lg, bad_L, mis):
+        assert f(*args) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_striped_featurize(p, p, p, p, p, p, 0, 2, 3, 100, 0, p, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_filter_exponential(p, p, 0, 3, 100, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_filter_exponential(p, p, 65, 3, 100, p, None) == hy.HYENA_ERR_INVALID_ARG
+    del ok

@@ -70,3 +70,21 @@ def test_linear_in_xq_and_in_hG_and_causal():
     y1 = oracle.striped_forward(xq, xk, xv, hT, hH, hK, hG)
     y2 = oracle.striped_forward(xq, xk, xv2, hT, hH, hK, hG)
     assert np.array_equal(y1[:, :t0], y2[:, :t0]) and not np.array_equal(y1[:, t0:], y2[:, t0:])
+
+
+def test_exponential_filter_matches_first_order_recurrences():
+    # conv with h_t = sum_n R_n lam_n^t equals the sum over n of the recurrences
+    # s_t = lam_n s_{t-1} + R_n z_t (the page's recurrent form of Hyena-LI)
+    L, d = 200, 3
+    R = rng.standard_normal((1, d))
+    lam = rng.uniform(-0.95, 0.95, (1, d))
+    z = rng.standard_normal(L)
+    h = oracle.exponential_filter(R, lam, L)[0]
+    ref = np.zeros(L)
+    for n in range(d):
+        s = 0.0
+        for t in range(L):
+            s = lam[0, n] * s + R[0, n] * z[t]
+            ref[t] += s
+    np.testing.assert_allclose(oracle.causal_conv(h, z, "direct"), ref, rtol=1e-10, atol=1e-12)
+    assert h[0] == pytest.approx(R.sum())
