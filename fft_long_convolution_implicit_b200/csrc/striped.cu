@@ -37,24 +37,84 @@ __device__ __forceinline__ void st1<float>(float* p, float v) { *p = v; }
 template <>
 __device__ __forceinline__ void st1<__nv_bfloat16>(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
 
-// s[i] = x[row + t0 - halo + i] as float, zero before t = 0 and from t = L on
+// Staged row: s[P + t - t0] = x[row + t] as float for t in [t0 - halo, t0 + n),
+// zero outside [0, L). P = padded halo (a multiple of 4), so the main part
+// starts on a 16-byte boundary; it is filled with 16-byte loads when the row
+// is suitably aligned (vec), else element by element.
 template <typename T>
-__device__ __forceinline__ void stage_row(float* s, const T* __restrict__ x, size_t row, int t0, int halo, int n, int L,
-                                          int tid) {
-  for (int i = tid; i < n; i += kStThreads) {
+__device__ __forceinline__ void stage_row(float* s, const T* __restrict__ x, size_t row, int t0, int halo, int P,
+                                          int n, int L, bool vec, int tid) {
+  for (int i = tid; i < halo; i += kStThreads) {
     const int t = t0 - halo + i;
-    s[i] = (t >= 0 && t < L) ? ld1<T>(x + row + t) : 0.f;
+    s[P - halo + i] = (t >= 0) ? ld1<T>(x + row + t) : 0.f;
+  }
+  constexpr int V = 16 / (int)sizeof(T);   // elements per 16-byte load
+  const int nv = vec ? n / V : 0;
+  for (int g = tid; g < nv; g += kStThreads) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + row + t0) + g);
+    float* d = s + P + g * V;
+    if constexpr (V == 8) {
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        d[2 * k] = __uint_as_float(w[k] << 16);
+        d[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+      }
+    } else {
+      *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                                  __uint_as_float(u.z), __uint_as_float(u.w));
+    }
+  }
+  for (int i = nv * V + tid; i < n; i += kStThreads) s[P + i] = ld1<T>(x + row + t0 + i);
+}
+
+__device__ __forceinline__ int pad4(int h) { return (h + 3) & ~3; }
+
+// acc[p] = sum_{j < len} f[j] s[P + base + p - j], p < kStPer, as a sliding
+// window over the staged row (positions below P - halo hold zeros or halo)
+__device__ __forceinline__ void fir8(const float* f, int len, const float* s, int pos, float (&acc)[kStPer]) {
+  float win[kStPer];
+#pragma unroll
+  for (int p = 0; p < kStPer; ++p) {
+    win[p] = s[pos + p];
+    acc[p] = 0.f;
+  }
+  for (int j = 0; j < len; ++j) {
+    const float g = f[j];
+#pragma unroll
+    for (int p = 0; p < kStPer; ++p) acc[p] = fmaf(g, win[p], acc[p]);
+#pragma unroll
+    for (int p = kStPer - 1; p > 0; --p) win[p] = win[p - 1];
+    if (j + 1 < len) win[0] = s[pos - j - 1];
   }
 }
 
-// Featurize q (optional) and u = (hH * xk)(hK * xv) for the rows' outputs.
+template <typename T>
+__device__ __forceinline__ void store8(T* dst, const float (&v)[kStPer]);
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* dst, const float (&v)[kStPer]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    w[k] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <>
+__device__ __forceinline__ void store8<float>(float* dst, const float (&v)[kStPer]) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// FUSED: y = q . (hG * u); otherwise q and u = k . v are written.
 template <typename T, bool FUSED>
 __global__ void __launch_bounds__(kStThreads)
 striped_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
                const float* __restrict__ hT, const float* __restrict__ hH, const float* __restrict__ hK, int lf,
                const float* __restrict__ hG, int lg, int D, int L, T* __restrict__ y, T* __restrict__ qout,
                T* __restrict__ uout) {
-  extern __shared__ float st[];
+  extern __shared__ __align__(16) float st[];
   const int tid = threadIdx.x;
   const int tiles = (L + kStTile - 1) / kStTile;
   const long long rowi = blockIdx.x / tiles;
@@ -62,19 +122,20 @@ striped_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __re
   const size_t row = (size_t)rowi * L;
   const int t0 = (int)(blockIdx.x % tiles) * kStTile;
   const int n_out = min(kStTile, L - t0);
-  const int hg = FUSED ? lg - 1 : 0;           // halo of u for the inner filter
-  const int hf = lf - 1;                        // halo of the featurizers
-  const int nu = n_out + hg;                    // u values this tile needs
-  const int nx = nu + hf;                       // xk, xv values
-  float* fT = st;                               // [lf]
+  const int hg = FUSED ? lg - 1 : 0;     // u halo for the inner filter
+  const int hf = lf - 1;                  // featurizer halo
+  const int Hx = hg + hf, Px = pad4(Hx);  // k, v rows
+  const int Pq = pad4(hf);                // q row
+  const int Pu = pad4(hg);                // u row
+  const int S = pad4(kStTile + lg + 24);  // capacity of each staged row (16-byte multiple)
+  float* fT = st;                         // [16]
   float* fH = fT + 16;
   float* fK = fH + 16;
-  float* fG = fK + 16;                          // [lg]
-  const int S = kStTile + lg + 16;              // staged-row capacity (>= nx)
-  float* sk = fG + (FUSED ? lg : 0);            // [nx]
+  float* fG = fK + 16;                    // [pad4(lg)]
+  float* sk = fG + (FUSED ? pad4(lg) : 0);
   float* sv = sk + S;
-  float* su = sv + S;                           // [nu]
-  float* sq = su + S;                           // [n_out + hf]
+  float* su = sv + S;
+  float* sq = su + S;
   for (int i = tid; i < lf; i += kStThreads) {
     fT[i] = hT[(size_t)c * lf + i];
     fH[i] = hH[(size_t)c * lf + i];
@@ -82,52 +143,61 @@ striped_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __re
   }
   if (FUSED)
     for (int i = tid; i < lg; i += kStThreads) fG[i] = hG[(size_t)c * lg + i];
-  stage_row<T>(sk, xk, row, t0, hg + hf, nx, L, tid);
-  stage_row<T>(sv, xv, row, t0, hg + hf, nx, L, tid);
-  stage_row<T>(sq, xq, row, t0, hf, n_out + hf, L, tid);
+  // rows of 16-byte multiples start 16-byte aligned: vector loads and stores
+  const bool vec = ((L * (int)sizeof(T)) & 15) == 0;
+  stage_row<T>(sk, xk, row, t0, Hx, Px, n_out, L, vec, tid);
+  stage_row<T>(sv, xv, row, t0, Hx, Px, n_out, L, vec, tid);
+  stage_row<T>(sq, xq, row, t0, hf, Pq, n_out, L, vec, tid);
   __syncthreads();
-  // u[i] = k . v at t = t0 - hg + i (zero before t = 0)
-  for (int i = tid; i < nu; i += kStThreads) {
+  const int base = tid * kStPer;
+  const bool full = base + kStPer <= n_out;
+  // u at t = t0 + base + p from the sliding windows; the halo t in [t0 - hg, t0) below
+  if (base < n_out) {
+    float a[kStPer], b[kStPer];
+    fir8(fH, lf, sk, Px + base, a);
+    fir8(fK, lf, sv, Px + base, b);
+#pragma unroll
+    for (int p = 0; p < kStPer; ++p) su[Pu + base + p] = a[p] * b[p];
+  }
+  for (int i = tid; i < hg; i += kStThreads) {
+    const int t = t0 - hg + i;
     float a = 0.f, b = 0.f;
     for (int j = 0; j < lf; ++j) {
-      a = fmaf(fH[j], sk[i + hf - j], a);
-      b = fmaf(fK[j], sv[i + hf - j], b);
+      a = fmaf(fH[j], sk[Px - hg + i - j], a);
+      b = fmaf(fK[j], sv[Px - hg + i - j], b);
     }
-    su[i] = (t0 - hg + i >= 0) ? a * b : 0.f;
+    su[Pu - hg + i] = t >= 0 ? a * b : 0.f;
   }
   __syncthreads();
-  // outputs t0 + base + p, p < kStPer
-  const int base = tid * kStPer;
   if (base >= n_out) return;
-  float acc[kStPer];
+  float q[kStPer];
+  fir8(fT, lf, sq, Pq + base, q);
+  float out[kStPer], u8[kStPer];
   if (FUSED) {
-    // inner sum w[t] = sum_j hG[j] u[t - j] as a sliding window: win[p] = u at (t_p - j)
+    fir8(fG, lg, su, Pu + base, out);
 #pragma unroll
-    for (int p = 0; p < kStPer; ++p) acc[p] = 0.f;
-    float win[kStPer];
+    for (int p = 0; p < kStPer; ++p) out[p] *= q[p];
+  } else {
 #pragma unroll
-    for (int p = 0; p < kStPer; ++p) win[p] = su[hg + base + p];   // j = 0
-    for (int j = 0; j < lg; ++j) {
-      const float g = fG[j];
-#pragma unroll
-      for (int p = 0; p < kStPer; ++p) acc[p] = fmaf(g, win[p], acc[p]);
-      // slide: index (base + p + hg) - (j + 1)
-#pragma unroll
-      for (int p = kStPer - 1; p > 0; --p) win[p] = win[p - 1];
-      win[0] = (j + 1 < lg) ? su[hg + base - j - 1] : 0.f;
-    }
+    for (int p = 0; p < kStPer; ++p) u8[p] = su[Pu + base + p];
   }
-#pragma unroll
-  for (int p = 0; p < kStPer; ++p) {
-    const int i = base + p;
-    if (i >= n_out) break;
-    float q = 0.f;
-    for (int j = 0; j < lf; ++j) q = fmaf(fT[j], sq[i + hf - j], q);
+  if (vec && full) {
     if (FUSED) {
-      st1<T>(y + row + t0 + i, q * acc[p]);
+      store8<T>(y + row + t0 + base, out);
     } else {
-      st1<T>(qout + row + t0 + i, q);
-      st1<T>(uout + row + t0 + i, su[i]);
+      store8<T>(qout + row + t0 + base, q);
+      store8<T>(uout + row + t0 + base, u8);
+    }
+  } else {
+#pragma unroll
+    for (int p = 0; p < kStPer; ++p) {
+      if (base + p >= n_out) break;
+      if (FUSED) {
+        st1<T>(y + row + t0 + base + p, out[p]);
+      } else {
+        st1<T>(qout + row + t0 + base + p, q[p]);
+        st1<T>(uout + row + t0 + base + p, u8[p]);
+      }
     }
   }
 }
@@ -145,7 +215,7 @@ __global__ void exp_sum_filter_kernel(const float* __restrict__ R, const float* 
 }
 
 size_t striped_smem(bool fused, int lg) {
-  return sizeof(float) * (size_t)(16 * 3 + (fused ? lg : 0) + 4 * (kStTile + lg + 16));
+  return sizeof(float) * (size_t)(16 * 3 + (fused ? ((lg + 3) & ~3) : 0) + 4 * ((kStTile + lg + 24 + 3) & ~3));
 }
 
 template <typename T, bool FUSED>
