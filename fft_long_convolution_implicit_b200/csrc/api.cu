@@ -180,9 +180,10 @@ const char* hyena_status_string(hyena_status s) {
 const char* hyena_last_cuda_error(void) { return g_last_cuda_error; }
 
 hyena_status hyena_device_timeouts(void) {
-  const int v = tc05_read_and_clear_timeout();
-  if (v < 0) return cuda_fail(cudaGetLastError());
-  return v ? HYENA_ERR_TIMEOUT : HYENA_OK;
+  const int a = tc05_read_and_clear_timeout();
+  const int b = striped_read_and_clear_timeout();
+  if (a < 0 || b < 0) return cuda_fail(cudaGetLastError());
+  return (a || b) ? HYENA_ERR_TIMEOUT : HYENA_OK;
 }
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {

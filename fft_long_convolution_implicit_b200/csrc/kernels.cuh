@@ -94,6 +94,7 @@ constexpr int kMaxStripedLG = 1024;
 cudaError_t launch_striped(const void* xq, const void* xk, const void* xv, const float* hT, const float* hH,
                            const float* hK, int lf, const float* hG, int lg, int B, int D, int L, bool bf16, void* y,
                            void* q, void* u, cudaStream_t s);
+int striped_read_and_clear_timeout();
 cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D, int L, float* h, cudaStream_t s);
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,

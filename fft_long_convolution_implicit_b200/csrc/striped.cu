@@ -202,6 +202,192 @@ striped_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __re
   }
 }
 
+// ---- persistent, bulk-copy-fed variant (rows of 16-byte multiples) ----------
+//
+// Work item = (row, tile of kStTile outputs). Each CTA walks items with a grid
+// stride; the three input windows [t0 - H, t0 + n) of item i + 1 are fetched
+// by one thread with cp.async.bulk (completion counted in bytes on the
+// stage's mbarrier) while item i is computed from the other stage. Inputs
+// stay in their storage type in shared memory; H is the causal halo rounded
+// up to 16 bytes (zeros are written there by the threads for t0 = 0).
+
+__device__ int g_striped_timeout;
+
+__device__ __forceinline__ uint32_t st_smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ bool st_mbar_wait(uint32_t bar, uint32_t phase) {
+  for (int it = 0; it < (1 << 24); ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+template <typename T>
+__device__ __forceinline__ float ldsT(const T* p);
+template <>
+__device__ __forceinline__ float ldsT<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ldsT<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// acc[p] = sum_{j < len} f[j] x[pos + p - j] over a staged row in storage type T
+template <typename T>
+__device__ __forceinline__ void fir8T(const float* f, int len, const T* x, int pos, float (&acc)[kStPer]) {
+  float win[kStPer];
+#pragma unroll
+  for (int p = 0; p < kStPer; ++p) {
+    win[p] = ldsT<T>(x + pos + p);
+    acc[p] = 0.f;
+  }
+  for (int j = 0; j < len; ++j) {
+    const float g = f[j];
+#pragma unroll
+    for (int p = 0; p < kStPer; ++p) acc[p] = fmaf(g, win[p], acc[p]);
+#pragma unroll
+    for (int p = kStPer - 1; p > 0; --p) win[p] = win[p - 1];
+    if (j + 1 < len) win[0] = ldsT<T>(x + pos - j - 1);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kStThreads)
+striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
+                    const float* __restrict__ hT, const float* __restrict__ hH, const float* __restrict__ hK, int lf,
+                    const float* __restrict__ hG, int lg, int D, int L, long long items, T* __restrict__ y) {
+  extern __shared__ __align__(128) unsigned char sraw[];
+  constexpr int E = (int)sizeof(T), V = 16 / E;
+  const int tid = threadIdx.x;
+  const int tiles = (L + kStTile - 1) / kStTile;
+  const int hg = lg - 1, hf = lf - 1, Hx = hg + hf;
+  const int HP = ((Hx + V - 1) / V) * V;           // halo slots, 16-byte multiple
+  const int W = HP + kStTile;                       // elements per staged window
+  const int Pu = pad4(hg);
+  const int S = pad4(kStTile + lg + 24);
+  const size_t winb = ((size_t)W * E + 127) & ~(size_t)127;
+  // [stage][xq, xk, xv] windows, then su (float), filters, mbarriers
+  float* su = reinterpret_cast<float*>(sraw + 6 * winb);
+  float* fT = su + S;
+  float* fH = fT + 16;
+  float* fK = fH + 16;
+  float* fG = fK + 16;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(fG + pad4(lg) + 4);
+  auto win = [&](int stage, int a) { return reinterpret_cast<T*>(sraw + (size_t)(3 * stage + a) * winb); };
+  const T* srcs[3] = {xq, xk, xv};
+
+  if (tid == 0) {
+    for (int k = 0; k < 2; ++k) asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(st_smem_u32(&bars[k])), "r"(1));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // one thread: expected bytes, then the three window copies of item it into stage
+  auto issue = [&](long long it, int stage) {
+    const long long rowi = it / tiles;
+    const int t0 = (int)(it % tiles) * kStTile;
+    const int n = min(kStTile, L - t0);
+    const int h = t0 >= HP ? HP : 0;               // first tile: halo zero-filled by the threads
+    const uint32_t bytes = (uint32_t)((h + n) * E);
+    const uint32_t bar = st_smem_u32(&bars[stage]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(3 * bytes) : "memory");
+    for (int a = 0; a < 3; ++a)
+      bulk_g2s(st_smem_u32(win(stage, a) + (HP - h)), srcs[a] + (size_t)rowi * L + t0 - h, bytes, bar);
+  };
+
+  uint32_t phase[2] = {0, 0};
+  bool pending[2] = {false, false};   // thread 0: a copy issued into the stage and not yet waited for
+  long long it = blockIdx.x;
+  if (tid == 0 && it < items) {
+    issue(it, 0);
+    pending[0] = true;
+  }
+  int stage = 0;
+  bool ok = true;
+  for (; it < items; it += gridDim.x, stage ^= 1) {
+    const long long rowi = it / tiles;
+    const int c = (int)(rowi % D);
+    const int t0 = (int)(it % tiles) * kStTile;
+    const int n_out = min(kStTile, L - t0);
+    // the other stage was released by the barrier that ended the last item
+    if (tid == 0 && it + gridDim.x < items) {
+      issue(it + gridDim.x, stage ^ 1);
+      pending[stage ^ 1] = true;
+    }
+    const bool done = st_mbar_wait(st_smem_u32(&bars[stage]), phase[stage]);
+    if (done) {
+      phase[stage] ^= 1;
+      pending[stage] = false;
+    } else if (tid == 0) {
+      atomicExch(&g_striped_timeout, 1);
+    }
+    const T* wq = win(stage, 0);
+    const T* wk = win(stage, 1);
+    const T* wv = win(stage, 2);
+    if (t0 < HP)
+      for (int i = tid; i < 3 * HP; i += kStThreads) win(stage, i / HP)[i % HP] = T(0.f);
+    for (int i = tid; i < lf; i += kStThreads) {
+      fT[i] = hT[(size_t)c * lf + i];
+      fH[i] = hH[(size_t)c * lf + i];
+      fK[i] = hK[(size_t)c * lf + i];
+    }
+    for (int i = tid; i < lg; i += kStThreads) fG[i] = hG[(size_t)c * lg + i];
+    ok = __syncthreads_and(done) != 0;
+    if (!ok) break;
+    // u = (hH * xk)(hK * xv) at t = t0 + base + p, and the halo t in [t0 - hg, t0)
+    const int base = tid * kStPer;
+    if (base < n_out) {
+      float a[kStPer], b[kStPer];
+      fir8T<T>(fH, lf, wk, HP + base, a);
+      fir8T<T>(fK, lf, wv, HP + base, b);
+#pragma unroll
+      for (int p = 0; p < kStPer; ++p) su[Pu + base + p] = a[p] * b[p];
+    }
+    for (int i = tid; i < hg; i += kStThreads) {
+      const int t = t0 - hg + i;
+      float a = 0.f, b = 0.f;
+      for (int j = 0; j < lf; ++j) {
+        a = fmaf(fH[j], ldsT<T>(wk + HP - hg + i - j), a);
+        b = fmaf(fK[j], ldsT<T>(wv + HP - hg + i - j), b);
+      }
+      su[Pu - hg + i] = t >= 0 ? a * b : 0.f;
+    }
+    __syncthreads();
+    if (base < n_out) {
+      float q[kStPer], out[kStPer];
+      fir8T<T>(fT, lf, wq, HP + base, q);
+      fir8(fG, lg, su, Pu + base, out);
+#pragma unroll
+      for (int p = 0; p < kStPer; ++p) out[p] *= q[p];
+      T* dst = y + (size_t)rowi * L + t0 + base;
+      if (base + kStPer <= n_out) {
+        store8<T>(dst, out);
+      } else {
+        for (int p = 0; p < kStPer && base + p < n_out; ++p) st1<T>(dst + p, out[p]);
+      }
+    }
+    // generic-proxy writes to this stage (halo zeros) before its next bulk copy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+  }
+  // after a timeout: wait (bounded) for the copies still in flight into this
+  // CTA's shared memory before it exits (normal exits leave none)
+  if (tid == 0)
+    for (int k = 0; k < 2; ++k)
+      if (pending[k]) st_mbar_wait(st_smem_u32(&bars[k]), phase[k]);
+  __syncthreads();
+}
+
 // h[c][t] = sum_n R[c][n] lambda[c][n]^t
 __global__ void exp_sum_filter_kernel(const float* __restrict__ R, const float* __restrict__ lam, int d, int D, int L,
                                       float* __restrict__ h) {
@@ -216,6 +402,31 @@ __global__ void exp_sum_filter_kernel(const float* __restrict__ R, const float* 
 
 size_t striped_smem(bool fused, int lg) {
   return sizeof(float) * (size_t)(16 * 3 + (fused ? ((lg + 3) & ~3) : 0) + 4 * ((kStTile + lg + 24 + 3) & ~3));
+}
+
+size_t striped_bulk_smem(int E, int lf, int lg) {
+  const int V = 16 / E, Hx = lg - 1 + lf - 1;
+  const size_t HP = (size_t)((Hx + V - 1) / V) * V;
+  const size_t winb = ((HP + kStTile) * E + 127) & ~(size_t)127;
+  const size_t S = (size_t)((kStTile + lg + 24 + 3) & ~3);
+  return 6 * winb + sizeof(float) * (S + 48 + (size_t)((lg + 3) & ~3) + 4) + 2 * sizeof(uint64_t);
+}
+
+template <typename T>
+cudaError_t launch_striped_bulk(const void* xq, const void* xk, const void* xv, const float* hT, const float* hH,
+                                const float* hK, int lf, const float* hG, int lg, int B, int D, int L, void* y,
+                                cudaStream_t s) {
+  auto k = striped_bulk_kernel<T>;
+  const size_t smem = striped_bulk_smem((int)sizeof(T), lf, lg);
+  int grid = 0;
+  cudaError_t e = persistent_grid((const void*)k, kStThreads, smem, &grid);
+  if (e != cudaSuccess) return e;
+  const long long items = (long long)((L + kStTile - 1) / kStTile) * B * D;
+  if ((long long)grid > items) grid = (int)items;
+  k<<<grid, kStThreads, smem, s>>>(reinterpret_cast<const T*>(xq), reinterpret_cast<const T*>(xk),
+                                   reinterpret_cast<const T*>(xv), hT, hH, hK, lf, hG, lg, D, L, items,
+                                   reinterpret_cast<T*>(y));
+  return cudaGetLastError();
 }
 
 template <typename T, bool FUSED>
@@ -240,11 +451,25 @@ cudaError_t launch_striped(const void* xq, const void* xk, const void* xv, const
                            const float* hK, int lf, const float* hG, int lg, int B, int D, int L, bool bf16, void* y,
                            void* q, void* u, cudaStream_t s) {
   const bool fused = (hG != nullptr);
+  // rows of 16-byte multiples: persistent kernel fed by bulk copies
+  if (fused && ((long long)L * (bf16 ? 2 : 4)) % 16 == 0)
+    return bf16 ? launch_striped_bulk<__nv_bfloat16>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, s)
+                : launch_striped_bulk<float>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, s);
   if (bf16)
     return fused ? launch_striped_t<__nv_bfloat16, true>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, q, u, s)
                  : launch_striped_t<__nv_bfloat16, false>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, q, u, s);
   return fused ? launch_striped_t<float, true>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, q, u, s)
                : launch_striped_t<float, false>(xq, xk, xv, hT, hH, hK, lf, hG, lg, B, D, L, y, q, u, s);
+}
+
+int striped_read_and_clear_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_striped_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_striped_timeout, &zero, sizeof(int));
+  }
+  return v;
 }
 
 cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D, int L, float* h, cudaStream_t s) {
