@@ -70,10 +70,12 @@ def tc05_built() -> bool:
     return hybuild.built_tc05()
 
 
-def dominant_kernel(w: synth.Workload) -> tuple[str, str]:
+def dominant_kernel(w: synth.Workload, spec16: bool = False) -> tuple[str, str]:
     """(kernel name, source set) of the launch that dominates one forward."""
     if w.L > 8192:
         return "four-step column/row kernels (whole step)", "fourstep"
+    if spec16:
+        return "fused_forward_kernel (f16 spectra)", "fused"
     if w.dtype == "bf16" and w.B % 2 == 0 and w.L == 2048 and tc05_built():
         return "tc05_forward_kernel", "tc05"
     if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
@@ -291,6 +293,8 @@ def main():
     ap.add_argument("--pass", dest="which", choices=["forward", "backward", "striped"], default="forward")
     ap.add_argument("--shape", default=None,
                     help="N,dtype,B,D,L: a custom shape instead of --config (small ncu captures)")
+    ap.add_argument("--spectrum", choices=["f32", "f16"], default="f32",
+                    help="forward pass: cached filter spectra as float32 (default) or f16 blocks")
     args = ap.parse_args()
     bwd = args.which == "backward"
     striped = args.which == "striped"
@@ -352,6 +356,9 @@ def main():
     base_v = torch.from_numpy(v_np).view(w.B, w.D, w.L).to(dev).to(dt)
     base_x = [torch.from_numpy(x).view(w.B, w.D, w.L).to(dev).to(dt) for x in xs_np]
     base_h = [hy.filter_rfft(h[n]) for n in range(w.N)]
+    spec16 = args.spectrum == "f16" and args.which == "forward"
+    if spec16:
+        base_h = [hy.spectrum_to_f16(t, w.D, w.L) for t in base_h]
     del h
     base_dy = (torch.from_numpy(synth.dy_rows(wr)).view(w.B, w.D, w.L).to(dev).to(dt) if bwd else None)
     set_bytes = ((w.N + 2 + (1 if bwd else 0)) * w.channels * w.L * w.elem_bytes
@@ -375,7 +382,7 @@ def main():
         if bwd:
             dv_, dxs_, dh_, ws_ = shared_out
             return hy.PreparedBackward(v_s, x_s, h_s, dy_s, dv=dv_, dxs=dxs_, dh=dh_, workspace=ws_, stream=st)
-        return hy.PreparedForward(v_s, x_s, h_s, stream=st)
+        return hy.PreparedForward(v_s, x_s, h_s, stream=st, f16_spectra=spec16)
 
     sets = []
     for s in range(nsets):
@@ -426,6 +433,9 @@ def main():
         alg_bytes = 4 * w.channels * w.L * w.elem_bytes + 4 * w.D * (3 * STRIPED_LF + STRIPED_LG)
     else:
         alg_bytes = w.roofline_bytes()
+        if spec16:
+            # the spectra are read as 4-byte f16 pairs instead of 8-byte float2
+            alg_bytes -= 4 * w.N * w.D * (w.L + 1)
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs in, result out
@@ -451,7 +461,7 @@ def main():
         d2h = w.channels * w.L * w.elem_bytes
     else:
         pin_y = torch.empty_like(pin_v).pin_memory()
-        e2e_call = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream)
+        e2e_call = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream, f16_spectra=spec16)
         h2d = (w.N + 1) * w.channels * w.L * w.elem_bytes
         d2h = w.channels * w.L * w.elem_bytes
 
@@ -491,15 +501,16 @@ def main():
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype, "pass": args.which,
+                       "spectra": "f16" if spec16 else "f32",
                        "global_batch": w.B * world, "parallelism": f"replicas x{world}",
                        "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
                              f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": None if (bwd or striped) else measured_traffic(w.name),
+                         "traffic": None if (bwd or striped or spec16) else measured_traffic(w.name),
                          "peak_kind": peak_kind, "alg_bytes_per_launch": alg_bytes,
                          "kernel": ("whole backward step (all its launches)" if bwd else
-                                    ("striped_kernel (fused FIR)" if striped else dominant_kernel(w)[0])),
+                                    ("striped_kernel (fused FIR)" if striped else dominant_kernel(w, spec16)[0])),
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},

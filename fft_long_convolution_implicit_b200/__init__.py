@@ -30,6 +30,7 @@ EXPORTS = (
     "hyena_abi_version", "hyena_forward_static_workspace", "hyena_backward_workspace_bytes", "hyena_backward",
     "hyena_filter_backward_workspace_bytes", "hyena_filter_backward", "hyena_device_timeouts",
     "hyena_striped_forward", "hyena_striped_featurize", "hyena_filter_exponential",
+    "hyena_filter_spectrum_bytes_f16", "hyena_filter_spectrum_to_f16", "hyena_forward_f16_spectra",
 )
 
 
@@ -75,6 +76,12 @@ def load() -> ctypes.CDLL:
     l.hyena_filter_rfft.restype = i
     l.hyena_spectrum_layout.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(i), ctypes.POINTER(i)]
     l.hyena_spectrum_layout.restype = i
+    l.hyena_filter_spectrum_bytes_f16.argtypes = [i, i]
+    l.hyena_filter_spectrum_bytes_f16.restype = sz
+    l.hyena_filter_spectrum_to_f16.argtypes = [P, i, i, P, P]
+    l.hyena_filter_spectrum_to_f16.restype = i
+    l.hyena_forward_f16_spectra.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
+    l.hyena_forward_f16_spectra.restype = i
     l.hyena_forward_workspace_bytes.argtypes = [i, i, i, i, i]
     l.hyena_forward_workspace_bytes.restype = sz
     l.hyena_forward.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
@@ -232,6 +239,46 @@ def forward(v, xs, hhats, y=None, workspace=None, stream=None):
     return y
 
 
+def spectrum_to_f16(hhat, D: int, L: int, hhat16=None, stream=None):
+    """f16 copy (uint8 CUDA tensor) of a float32 spectrum block from filter_rfft."""
+    torch = _torch()
+    nbytes = load().hyena_filter_spectrum_bytes_f16(D, L)
+    if nbytes == 0:
+        _check(HYENA_ERR_UNSUPPORTED, "hyena_filter_spectrum_bytes_f16")
+    if hhat.numel() * hhat.element_size() < filter_spectrum_bytes(D, L):
+        raise ValueError("hhat is smaller than a float32 spectrum block for (D, L)")
+    if hhat16 is None:
+        hhat16 = torch.empty(nbytes, dtype=torch.uint8, device=hhat.device)
+    _check(load().hyena_filter_spectrum_to_f16(_dev(hhat, "hhat"), D, L, _dev(hhat16, "hhat16"), _stream(stream)),
+           "hyena_filter_spectrum_to_f16")
+    return hhat16
+
+
+def forward_f16_spectra(v, xs, hhats16, y=None, workspace=None, stream=None):
+    """forward() with f16 spectrum blocks from spectrum_to_f16."""
+    torch = _torch()
+    B, D, L = v.shape
+    N = len(xs)
+    if len(hhats16) != N:
+        raise ValueError("need one spectrum per gate")
+    code = _dtype_code(v)
+    for x in xs:
+        if x.shape != v.shape or x.dtype != v.dtype:
+            raise ValueError("gates must match v in shape and dtype")
+    if y is None:
+        y = torch.empty_like(v)
+    ws_need = forward_workspace_bytes(B, D, L, N, code == HYENA_BF16)
+    if workspace is None and ws_need:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=v.device)
+    xarr = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+    harr = (ctypes.c_void_p * N)(*[_dev(hh, "hhat16").value for hh in hhats16])
+    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else ctypes.c_void_p(0)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().hyena_forward_f16_spectra(_dev(v, "v"), xarr, harr, B, D, L, N, code, _dev(y, "y"), ws_ptr,
+                                            ws_bytes, _stream(stream)), "hyena_forward_f16_spectra")
+    return y
+
+
 def forward_static_workspace(v, xs, hhats, y=None, stream=None):
     """hyena_forward_static_workspace: the long-sequence forward (8192 < L)
     with the library's static device scratch instead of a caller workspace,
@@ -327,9 +374,11 @@ def spectrum_natural(hhat, D: int, L: int):
 class PreparedForward:
     """hyena_forward with its arguments marshalled once (fixed tensors and
     stream); calling it issues the C call only. Keeps host overhead per
-    call to a few microseconds for back-to-back launches."""
+    call to a few microseconds for back-to-back launches. With
+    f16_spectra=True, hhats are f16 blocks (spectrum_to_f16) and the call is
+    hyena_forward_f16_spectra."""
 
-    def __init__(self, v, xs, hhats, y=None, workspace=None, stream=None):
+    def __init__(self, v, xs, hhats, y=None, workspace=None, stream=None, f16_spectra: bool = False):
         torch = _torch()
         B, D, L = v.shape
         N = len(xs)
@@ -345,12 +394,13 @@ class PreparedForward:
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
         self._args = (_dev(v, "v"), self._x, self._h, B, D, L, N, code, _dev(self.y, "y"), ws_ptr, ws_bytes,
                       _stream(stream))
-        self._fn = load().hyena_forward
+        self._name = "hyena_forward_f16_spectra" if f16_spectra else "hyena_forward"
+        self._fn = getattr(load(), self._name)
 
     def __call__(self):
         st = self._fn(*self._args)
         if st != HYENA_OK:
-            raise HyenaError(st, "hyena_forward")
+            raise HyenaError(st, self._name)
         return self.y
 
 

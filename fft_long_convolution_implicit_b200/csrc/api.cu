@@ -84,8 +84,11 @@ cudaError_t hyena::persistent_grid(const void* kernel, int threads, size_t smem,
 
 cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const void* const* hhat, int B, int D,
                                     const Layout& ly, int N, bool bf16, void* y, void* workspace,
-                                    size_t workspace_bytes, bool allow_tc, cudaStream_t s) {
-  const float2* tables = reinterpret_cast<const float2*>(hhat[0]) + tables_offset(ly, D);
+                                    size_t workspace_bytes, bool allow_tc, cudaStream_t s, bool spec16) {
+  const float2* tables =
+      spec16 ? reinterpret_cast<const float2*>(reinterpret_cast<const char*>(hhat[0]) + spec16_tables_offset_bytes(ly, D))
+             : reinterpret_cast<const float2*>(hhat[0]) + tables_offset(ly, D);
+  if (spec16) allow_tc = false;   // the tensor-core kernels read their own float32 copy
   cudaError_t e = cudaSuccess;
   if (!ly.fourstep) {
     FusedLaunch p{};
@@ -98,6 +101,7 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     p.tables = tables;
     p.B = B; p.D = D; p.L = ly.L; p.N = N;
     p.bf16 = bf16;
+    p.spec16 = spec16;
     if (allow_tc && ly.tc && p.bf16 && (B % 2) == 0) {
       // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
       for (int n = 0; n < N; ++n)
@@ -124,6 +128,7 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     p.scratch = reinterpret_cast<float2*>(workspace);
     p.B = B; p.D = D; p.L = ly.L; p.N = N;
     p.bf16 = bf16;
+    p.spec16 = spec16;
     for (long long c0 = 0; c0 < C && e == cudaSuccess; c0 += w) {
       p.ch0 = c0;
       p.wave = (int)((C - c0) < w ? (C - c0) : w);
@@ -246,6 +251,39 @@ hyena_status hyena_forward(const void* v, const void* const* x, const void* cons
     return HYENA_ERR_WORKSPACE;
   const cudaError_t e = forward_dispatch(v, x, hhat, B, D, ly, N, dtype == HYENA_BF16, y, workspace,
                                          workspace_bytes, true, (cudaStream_t)stream);
+  return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
+}
+
+size_t hyena_filter_spectrum_bytes_f16(int D, int L) {
+  Layout y;
+  if (D < 1 || !make_layout(L, &y)) return 0;
+  return spec16_block_bytes(y, D);
+}
+
+hyena_status hyena_filter_spectrum_to_f16(const void* hhat, int D, int L, void* hhat16, hyena_stream stream) {
+  if (!aligned16(hhat) || !aligned16(hhat16) || D < 1) return HYENA_ERR_INVALID_ARG;
+  Layout y;
+  if (!make_layout(L, &y)) return HYENA_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_spectrum_to_f16(reinterpret_cast<const float2*>(hhat),
+                                               reinterpret_cast<unsigned char*>(hhat16), D, y, (cudaStream_t)stream);
+  return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
+}
+
+hyena_status hyena_forward_f16_spectra(const void* v, const void* const* x, const void* const* hhat16, int B, int D,
+                                       int L, int N, hyena_dtype dtype, void* y, void* workspace,
+                                       size_t workspace_bytes, hyena_stream stream) {
+  if (N < 1 || N > kMaxOrder || B < 1 || D < 1) return HYENA_ERR_INVALID_ARG;
+  if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+  if (!x || !hhat16 || !aligned16(v) || !aligned16(y)) return HYENA_ERR_INVALID_ARG;
+  for (int n = 0; n < N; ++n)
+    if (!aligned16(x[n]) || !aligned16(hhat16[n])) return HYENA_ERR_INVALID_ARG;
+  if ((long long)B * D > (1LL << 40) / (L > 0 ? L : 1)) return HYENA_ERR_INVALID_ARG;
+  Layout ly;
+  if (!make_layout(L, &ly)) return HYENA_ERR_UNSUPPORTED;
+  if (ly.fourstep && (!aligned16(workspace) || workspace_bytes < sizeof(float2) * (size_t)ly.M))
+    return HYENA_ERR_WORKSPACE;
+  const cudaError_t e = forward_dispatch(v, x, hhat16, B, D, ly, N, dtype == HYENA_BF16, y, workspace,
+                                         workspace_bytes, false, (cudaStream_t)stream, true);
   return e == cudaSuccess ? HYENA_OK : cuda_fail(e);
 }
 

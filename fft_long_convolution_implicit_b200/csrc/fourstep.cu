@@ -42,7 +42,8 @@ __device__ __forceinline__ float2 expi_neg(int e, int M) {
 template <int MB, int MODE, typename T>
 __global__ void __launch_bounds__(ColCfg<MB>::THREADS)
 col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict__ yout, float2* __restrict__ scr,
-           const float2* __restrict__ tw1, int B, int D, int L, int MV, long long ch0) {
+           const float2* __restrict__ tw1, int B, int D, int L, int MV, long long ch0,
+           const float* __restrict__ inv_scale) {
   using Cfg = ColCfg<MB>;
   constexpr int M1 = Cfg::M1, CW = Cfg::CW, NQ = 16 / MB;
   extern __shared__ float2 sm[];
@@ -85,11 +86,13 @@ col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict_
       for (int r = 0; r < 16; ++r) a[r] = csm[pidx(16 * j + r)];
     }
     dft16<true, false, true, 0>(a);          // outputs n1 = j + r*MB, r < 8
+    // reduced-precision spectra: the channel's exact inverse scale joins the gate
+    const float inv = inv_scale ? __ldg(inv_scale + c) : 1.f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const size_t m = (size_t)MV * (j + r * MB) + n2;
       const float2 g = IO<T>::load2_stream(gate + row + 2 * m);
-      a[r] = make_float2(a[r].x * g.x, a[r].y * g.y);
+      a[r] = make_float2(a[r].x * (g.x * inv), a[r].y * (g.y * inv));
     }
     if constexpr (MODE == kColLast) {
 #pragma unroll
@@ -135,7 +138,7 @@ constexpr int row_blocks() {
   return 512 / (2 * Plan<LOGMV>::TV) > 1 ? 512 / (2 * Plan<LOGMV>::TV) : 1;
 }
 
-template <int LOGMV, int MODE>
+template <int LOGMV, int MODE, typename HT = float2>
 __global__ void __launch_bounds__(2 * Plan<LOGMV>::TV, row_blocks<LOGMV>())
 row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const float2* __restrict__ tables, int M1,
            int B, long long ch0) {
@@ -147,15 +150,13 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
   const float2* __restrict__ Wv = tables + MV;
   const int p = blockIdx.x;
   const int kA = p, kB = (p == 0) ? M1 / 2 : M1 - p;
-  float2* S;
-  float2* H;
-  if (MODE == kPairConv) {
-    S = scr + (size_t)blockIdx.y * M;
+  float2* S = scr + (size_t)blockIdx.y * M;
+  HT* H;
+  if constexpr (MODE == kPairConv) {
     const long long ch = ch0 + blockIdx.y;
-    H = const_cast<float2*>(spec) + (size_t)(ch / B) * M;
+    H = reinterpret_cast<HT*>(const_cast<float2*>(spec)) + (size_t)(ch / B) * M;
   } else {
-    S = scr + (size_t)blockIdx.y * M;   // spectrum block of channel blockIdx.y, transformed in place
-    H = S;
+    H = S;   // spectrum block of channel blockIdx.y, transformed in place
   }
   const int t = threadIdx.x;
   const int vec = t / TV, tl = t % TV;
@@ -183,7 +184,8 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
   mid_fwd_all<LOGMV>(a, base, tw, tl);
 
   {
-    float2 *bA, *bB, *HA, *HB;
+    float2 *bA, *bB;
+    HT *HA, *HB;
     int jA, jB;
     bool head = false, has_rho = true;
     float2 rho;
@@ -209,7 +211,7 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
       rho = make_float2(c, -s);
       HA = HB = H + (size_t)(M1 / 2) * MV;
     }
-    paired_pass<LOGMV, MODE>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
+    paired_pass<LOGMV, MODE, false, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
   }
   if (MODE == kPairSpectrum) return;
   __syncthreads();
@@ -238,20 +240,21 @@ static cudaError_t prep(K kernel, size_t smem) {
 
 template <int MB, int MODE, typename T>
 static cudaError_t launch_col(const T* zin, const T* gate, T* yout, float2* scr, const float2* tw1, int B, int D,
-                              int L, int MV, long long ch0, int nch, cudaStream_t s) {
+                              int L, int MV, long long ch0, int nch, cudaStream_t s,
+                              const float* inv_scale = nullptr) {
   using Cfg = ColCfg<MB>;
   auto k = col_kernel<MB, MODE, T>;
   cudaError_t e = prep(k, Cfg::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid(MV / Cfg::CW, nch);
-  k<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(zin, gate, yout, scr, tw1, B, D, L, MV, ch0);
+  k<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(zin, gate, yout, scr, tw1, B, D, L, MV, ch0, inv_scale);
   return cudaGetLastError();
 }
 
-template <int LOGMV, int MODE>
+template <int LOGMV, int MODE, typename HT = float2>
 static cudaError_t launch_row(float2* scr, const float2* spec, const float2* tables, int M1, int B, long long ch0,
                               int nch, cudaStream_t s) {
-  auto k = row_kernel<LOGMV, MODE>;
+  auto k = row_kernel<LOGMV, MODE, HT>;
   const size_t smem = sizeof(float2) * 2 * (size_t)padded_len(1 << LOGMV);
   cudaError_t e = prep(k, smem);
   if (e != cudaSuccess) return e;
@@ -260,28 +263,33 @@ static cudaError_t launch_row(float2* scr, const float2* spec, const float2* tab
   return cudaGetLastError();
 }
 
-template <int LOGMV, int MB, typename T>
+template <int LOGMV, int MB, typename T, typename HT>
 static cudaError_t wave_t(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
   const float2* tw1 = p.tables + y.tw_1;
   const int MV = y.MV;
   cudaError_t e = launch_col<MB, kColFirst, T>(reinterpret_cast<const T*>(p.v), nullptr, nullptr, p.scratch, tw1,
                                                p.B, p.D, p.L, MV, p.ch0, p.wave, s);
   for (int n = 0; n < p.N && e == cudaSuccess; ++n) {
-    e = launch_row<LOGMV, kPairConv>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);
+    e = launch_row<LOGMV, kPairConv, HT>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);
     if (e != cudaSuccess) break;
+    const float* inv = nullptr;
+    if (sizeof(HT) != sizeof(float2))
+      inv = reinterpret_cast<const float*>(reinterpret_cast<const char*>(p.hh.p[n]) + spec16_scales_offset_bytes(y, p.D));
     const T* g = reinterpret_cast<const T*>(p.x[n]);
     if (n + 1 < p.N)
-      e = launch_col<MB, kColMid, T>(nullptr, g, nullptr, p.scratch, tw1, p.B, p.D, p.L, MV, p.ch0, p.wave, s);
+      e = launch_col<MB, kColMid, T>(nullptr, g, nullptr, p.scratch, tw1, p.B, p.D, p.L, MV, p.ch0, p.wave, s, inv);
     else
       e = launch_col<MB, kColLast, T>(nullptr, g, reinterpret_cast<T*>(p.y), p.scratch, tw1, p.B, p.D, p.L, MV,
-                                      p.ch0, p.wave, s);
+                                      p.ch0, p.wave, s, inv);
   }
   return e;
 }
 
 template <int LOGMV, int MB>
 static cudaError_t wave_lm(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
-  return p.bf16 ? wave_t<LOGMV, MB, __nv_bfloat16>(p, y, s) : wave_t<LOGMV, MB, float>(p, y, s);
+  if (p.spec16)
+    return p.bf16 ? wave_t<LOGMV, MB, __nv_bfloat16, __half2>(p, y, s) : wave_t<LOGMV, MB, float, __half2>(p, y, s);
+  return p.bf16 ? wave_t<LOGMV, MB, __nv_bfloat16, float2>(p, y, s) : wave_t<LOGMV, MB, float, float2>(p, y, s);
 }
 
 template <int LOGMV>

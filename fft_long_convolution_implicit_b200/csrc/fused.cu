@@ -24,26 +24,37 @@ struct FusedOcc {
   static constexpr int value = TV >= 512 ? 1 : (T / TV > 16 ? 16 : (T / TV < 1 ? 1 : T / TV));
 };
 
-// Shared memory: z (padded), staged filter spectrum row, staged gate row,
-// staged v row of the next channel.
-template <int LOGMV, typename T>
+// Shared memory: z (padded), staged filter spectrum row (bins of type HT),
+// staged gate row, staged v row of the next channel.
+template <int LOGMV, typename T, typename HT = float2>
 struct FusedSmem {
   static constexpr int MV = 1 << LOGMV;
   static constexpr size_t z = sizeof(float2) * padded_len(MV);
-  static constexpr size_t h = sizeof(float2) * MV;
+  static constexpr size_t h = sizeof(HT) * MV;
   static constexpr size_t row = sizeof(T) * MV;      // L <= MV elements, 16-byte multiple
   static constexpr size_t total = z + h + 2 * row;
 };
 
-template <int LOGMV, typename T>
+// Per-channel factor of a spectrum block: 1 for float32 bins; for __half2
+// bins the inverse of the channel's power-of-two scale (exact), applied at the gate.
+template <typename HT>
+__device__ __forceinline__ float spec_inv_scale(const float2* block, int D, int M, int c) {
+  if constexpr (sizeof(HT) == sizeof(float2)) {
+    return 1.f;
+  } else {
+    return __ldg(reinterpret_cast<const float*>(reinterpret_cast<const char*>(block) + (size_t)4 * D * M) + c);
+  }
+}
+
+template <int LOGMV, typename T, typename HT>
 __global__ void __launch_bounds__(Plan<LOGMV>::TV, FusedOcc<LOGMV>::value)
 fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __restrict__ y,
                      const float2* __restrict__ tables, int B, int D, int L, int N) {
   using P = Plan<LOGMV>;
-  using S = FusedSmem<LOGMV, T>;
+  using S = FusedSmem<LOGMV, T, HT>;
   constexpr int MV = P::MV, TV = P::TV, Q8 = MV / 8, Q16 = MV / 16;
   extern __shared__ __align__(16) float2 sm[];
-  float2* hs = reinterpret_cast<float2*>(reinterpret_cast<char*>(sm) + S::z);
+  HT* hs = reinterpret_cast<HT*>(reinterpret_cast<char*>(sm) + S::z);
   T* xs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h);
   T* vs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h + S::row);
   const int tl = threadIdx.x;
@@ -55,14 +66,15 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
   const int jB = head ? Q16 : Q8 - tl;
   const float2 one = make_float2(1.f, 0.f);
   const int row_bytes = L * (int)sizeof(T);
-  const int h_bytes = MV * (int)sizeof(float2);
+  const int h_bytes = MV * (int)sizeof(HT);
+  auto spec_row = [&](int n, int c) { return reinterpret_cast<const HT*>(pick(hh, n)) + (size_t)c * MV; };
 
   // channel order c-major so that CTAs sharing a filter run side by side
   long long ch = blockIdx.x;
   if (ch < C) {
     const int c = (int)(ch / B), b = (int)(ch % B);
     block_copy_async(vs, v + ((size_t)b * D + c) * (size_t)L, row_bytes, tl, TV);
-    block_copy_async(hs, pick(hh, 0) + (size_t)c * MV, h_bytes, tl, TV);
+    block_copy_async(hs, spec_row(0, c), h_bytes, tl, TV);
     cp_async_commit();
     cp_async_wait_all();
   }
@@ -95,15 +107,15 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
       cp_async_wait_all();
       __syncthreads();
       // last forward pass + spectral product + first inverse pass
-      paired_pass<LOGMV, kPairConv, true>(sm, sm, jA, jB, head, tw, Wv, one, false, hs, hs, 0.f);
+      paired_pass<LOGMV, kPairConv, true, HT>(sm, sm, jA, jB, head, tw, Wv, one, false, hs, hs, 0.f);
       __syncthreads();
       // the spectrum buffer is free: stage the next spectrum (next stage or next channel)
       {
-        const float2* hn = nullptr;
+        const HT* hn = nullptr;
         if (n + 1 < N) {
-          hn = pick(hh, n + 1) + (size_t)c * MV;
+          hn = spec_row(n + 1, c);
         } else if (ch + gridDim.x < C) {
-          hn = pick(hh, 0) + (size_t)((ch + gridDim.x) / B) * MV;
+          hn = spec_row(0, (int)((ch + gridDim.x) / B));
         }
         if (hn) block_copy_async(hs, hn, h_bytes, tl, TV);
         cp_async_commit();
@@ -112,12 +124,13 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
       // last inverse pass (radix 16): only the first half of the outputs is kept
       load_block16(sm, tl, a);
       dft16<true, false, true, 0>(a);
-      // gate: z_{n+1}[t] = x_n[t] * conv[t]
+      // gate: z_{n+1}[t] = x_n[t] * conv[t] (times the spectrum block's channel factor)
+      const float inv = spec_inv_scale<HT>(pick(hh, n), D, MV, c);
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
         const int m = tl + r * Q16;
         const float2 g = (2 * m < L) ? IO<T>::load2_smem(xs + 2 * m) : make_float2(0.f, 0.f);
-        a[r] = make_float2(a[r].x * g.x, a[r].y * g.y);
+        a[r] = make_float2(a[r].x * (g.x * inv), a[r].y * (g.y * inv));
       }
     }
 #pragma unroll
@@ -165,11 +178,11 @@ fused_spectrum_kernel(const float* __restrict__ h, float2* __restrict__ spec, co
 
 // ------------------------------------------------------------- launchers --
 
-template <int LOGMV, typename T>
+template <int LOGMV, typename T, typename HT>
 static cudaError_t launch_fused_t(const FusedLaunch& p, cudaStream_t s) {
-  auto k = fused_forward_kernel<LOGMV, T>;
+  auto k = fused_forward_kernel<LOGMV, T, HT>;
   const int threads = Plan<LOGMV>::TV;
-  const size_t smem = FusedSmem<LOGMV, T>::total;
+  const size_t smem = FusedSmem<LOGMV, T, HT>::total;
   int grid = 0;
   cudaError_t e = persistent_grid((const void*)k, threads, smem, &grid);
   if (e != cudaSuccess) return e;
@@ -184,7 +197,9 @@ static cudaError_t launch_fused_t(const FusedLaunch& p, cudaStream_t s) {
 
 template <int LOGMV>
 static cudaError_t launch_fused_l(const FusedLaunch& p, cudaStream_t s) {
-  return p.bf16 ? launch_fused_t<LOGMV, __nv_bfloat16>(p, s) : launch_fused_t<LOGMV, float>(p, s);
+  if (p.spec16)
+    return p.bf16 ? launch_fused_t<LOGMV, __nv_bfloat16, __half2>(p, s) : launch_fused_t<LOGMV, float, __half2>(p, s);
+  return p.bf16 ? launch_fused_t<LOGMV, __nv_bfloat16, float2>(p, s) : launch_fused_t<LOGMV, float, float2>(p, s);
 }
 
 cudaError_t launch_fused_forward(const FusedLaunch& p, int logMV, cudaStream_t s) {

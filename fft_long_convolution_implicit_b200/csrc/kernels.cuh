@@ -40,6 +40,7 @@ struct FusedLaunch {
   const float2* tables;
   int B, D, L, N;
   bool bf16;
+  bool spec16;       // spectrum blocks in the reduced-precision (__half2) format
 };
 
 struct FourStepLaunch {
@@ -53,6 +54,7 @@ struct FourStepLaunch {
   bool bf16;
   long long ch0;     // first channel (c-major order) of this wave
   int wave;          // channels in this wave
+  bool spec16;       // spectrum blocks in the reduced-precision (__half2) format
 };
 
 // Records e as this thread's last CUDA error (hyena_last_cuda_error) and
@@ -64,7 +66,9 @@ hyena_status report_cuda_error(cudaError_t e);
 // Arguments are assumed checked by the caller.
 cudaError_t forward_dispatch(const void* v, const void* const* x, const void* const* hhat, int B, int D,
                              const Layout& ly, int N, bool bf16, void* y, void* workspace, size_t workspace_bytes,
-                             bool allow_tc, cudaStream_t s);
+                             bool allow_tc, cudaStream_t s, bool spec16 = false);
+// float32 spectrum block -> reduced-precision block (bins and scales; tables copied)
+cudaError_t launch_spectrum_to_f16(const float2* spec, unsigned char* out, int D, const Layout& y, cudaStream_t s);
 // Workspace of one L2-sized four-step wave over `channels` channels.
 size_t fourstep_wave_bytes(long long channels, const Layout& ly);
 // Spectrum block (spectra, optional tensor-core copy, tables) of `rows` real

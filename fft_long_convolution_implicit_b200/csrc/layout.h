@@ -94,4 +94,13 @@ inline size_t tables_offset(const Layout& y, int D) {
 }
 inline size_t spectrum_block_floats2(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
 
+// Reduced-precision spectrum block: [D][M] __half2 bins (same order, each
+// channel scaled by a power of two), [D] float 1 / scale (padded to 16 bytes),
+// then the same table region as the float32 block.
+inline size_t spec16_scales_offset_bytes(const Layout& y, int D) { return (size_t)4 * D * y.M; }
+inline size_t spec16_tables_offset_bytes(const Layout& y, int D) {
+  return ((size_t)4 * D * y.M + (size_t)4 * D + 15) & ~(size_t)15;
+}
+inline size_t spec16_block_bytes(const Layout& y, int D) { return spec16_tables_offset_bytes(y, D) + 8 * (size_t)y.table_len; }
+
 }  // namespace hyena

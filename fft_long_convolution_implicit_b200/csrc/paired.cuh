@@ -9,6 +9,8 @@
 // head thread of row 0, whose butterflies 0 and MV/16 are each self-mirrored.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "fft_engine.cuh"
 
 namespace hyena {
@@ -16,16 +18,26 @@ namespace hyena {
 enum PairMode { kPairConv = 0, kPairSpectrum = 1 };
 
 // Filter spectrum reads: from global memory through the read-only path, or
-// from a shared-memory copy staged by the caller (H_SMEM).
-template <bool H_SMEM>
+// from a shared-memory copy staged by the caller (H_SMEM); bins stored as
+// float2, or as __half2 (the reduced-precision block, scaled per channel by
+// a power of two that the caller removes at the gate).
+template <bool H_SMEM, typename HT = float2>
 struct HRead;
 template <>
-struct HRead<false> {
+struct HRead<false, float2> {
   static __device__ __forceinline__ float2 at(const float2* p, int i) { return __ldg(p + i); }
 };
 template <>
-struct HRead<true> {
+struct HRead<true, float2> {
   static __device__ __forceinline__ float2 at(const float2* p, int i) { return p[i]; }
+};
+template <>
+struct HRead<false, __half2> {
+  static __device__ __forceinline__ float2 at(const __half2* p, int i) { return __half22float2(__ldg(p + i)); }
+};
+template <>
+struct HRead<true, __half2> {
+  static __device__ __forceinline__ float2 at(const __half2* p, int i) { return __half22float2(p[i]); }
 };
 
 // W for bin kA of row A: w_{2M}^{k1 + M1 k2} = rho * w_{2 MV}^{k2}.
@@ -39,12 +51,13 @@ __device__ __forceinline__ float2 pair_w(const float2* __restrict__ Wv, int k2, 
 // MODE kPairSpectrum: the unpacked spectrum 2 Z[k] * scale is written to HA/HB
 //   (library order, packed DC/Nyquist in bin 0 of row 0); shared memory is not
 //   written back.
-template <int LOGMV, int MODE, bool H_SMEM = false>
+template <int LOGMV, int MODE, bool H_SMEM = false, typename HT = float2>
 __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA, int jB, bool head,
                                             const float2* __restrict__ tw, const float2* __restrict__ Wv,
-                                            float2 rho, bool has_rho, float2* HA, float2* HB, float scale) {
+                                            float2 rho, bool has_rho, HT* HA, HT* HB, float scale) {
   constexpr int MV = 1 << LOGMV, Q8 = MV / 8, Q16 = MV / 16, NS = Q8;
-  auto hload = [](const float2* p, int i) { return HRead<H_SMEM>::at(p, i); };
+  static_assert(MODE == kPairConv || sizeof(HT) == sizeof(float2), "spectra are written as float2");
+  auto hload = [](const HT* p, int i) { return HRead<H_SMEM, HT>::at(p, i); };
   float2 a[8], b[8];
   float2* pa = baseA + pidx(jA);
   float2* pb = baseB + pidx(jB);
@@ -70,7 +83,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     for (int r = 0; r < 8; ++r) {
       const int kA = jA + r * Q8;
       const float2 W = pair_w(Wv, kA, rho, has_rho);
-      if (MODE == kPairConv) {
+      if constexpr (MODE == kPairConv) {
         spectral_pair(a[r], b[7 - r], hload(HA, kA), hload(HB, jB + (7 - r) * Q8), W);
       } else {
         float2 za, zb;
@@ -84,7 +97,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     // bin M/2 with itself, and r with 8-r otherwise.
     {
       const float2 one = make_float2(1.f, 0.f);
-      if (MODE == kPairConv) {
+      if constexpr (MODE == kPairConv) {
         float2 c0 = a[0], c0b = a[0];
         const float2 h0 = hload(HA, 0);
         spectral_pair(c0, c0b, make_float2(h0.x, 0.f), make_float2(h0.y, 0.f), one);
@@ -98,7 +111,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
 #pragma unroll
     for (int r = 1; r < 4; ++r) {
       const float2 W = __ldg(&Wv[r * Q8]);
-      if (MODE == kPairConv) {
+      if constexpr (MODE == kPairConv) {
         spectral_pair(a[r], a[8 - r], hload(HA, r * Q8), hload(HA, (8 - r) * Q8), W);
       } else {
         float2 za, zb;
@@ -109,7 +122,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     }
     {
       const float2 W = __ldg(&Wv[4 * Q8]);
-      if (MODE == kPairConv) {
+      if constexpr (MODE == kPairConv) {
         float2 c4 = a[4], c4b = a[4];
         const float2 h4 = hload(HA, 4 * Q8);
         spectral_pair(c4, c4b, h4, h4, W);
@@ -124,7 +137,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float2 W = __ldg(&Wv[Q16 + r * Q8]);
-      if (MODE == kPairConv) {
+      if constexpr (MODE == kPairConv) {
         spectral_pair(b[r], b[7 - r], hload(HA, Q16 + r * Q8), hload(HA, Q16 + (7 - r) * Q8), W);
       } else {
         float2 za, zb;
@@ -135,7 +148,7 @@ __device__ __forceinline__ void paired_pass(float2* baseA, float2* baseB, int jA
     }
   }
 
-  if (MODE == kPairConv) {
+  if constexpr (MODE == kPairConv) {
     dft8<true, 0>(a);
     dft8<true, 0>(b);
 #pragma unroll

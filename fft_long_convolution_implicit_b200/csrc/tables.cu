@@ -5,6 +5,8 @@
 //  w_v[k]:  w_{2 MV}^k, k < MV (real-FFT unpack twiddle of the row transform).
 //  tw_1[i]: twiddles of the M1-point column plan (radix 16, then radix M1/16).
 // Values are formed in double with sincospi and rounded once to float.
+#include <cuda_fp16.h>
+
 #include "kernels.cuh"
 
 namespace hyena {
@@ -69,6 +71,46 @@ cudaError_t launch_fill_tables(float2* tables, const Layout& y, cudaStream_t s) 
   fill_tables_kernel<<<(n + 255) / 256, 256, 0, s>>>(tables, pv, p1, y.MV, y.fourstep ? y.M1 : 0, y.tw_v, y.w_v,
                                                      y.tw_1, y.table_len);
   return cudaGetLastError();
+}
+
+}  // namespace hyena
+
+namespace hyena {
+
+// Reduced-precision copy of a spectrum block, one CTA per channel: bins as
+// __half2 after multiplying by the power of two f_c that brings every
+// component below 2^15 (the f16 range stops at 65504), and 1 / f_c per channel.
+__global__ void spectrum_to_f16_kernel(const float2* __restrict__ spec, __half2* __restrict__ out,
+                                       float* __restrict__ inv_scale, int M) {
+  __shared__ float red[8];
+  const int c = blockIdx.x, tid = threadIdx.x;
+  const float2* __restrict__ row = spec + (size_t)c * M;
+  float mx = 0.f;
+  for (int i = tid; i < M; i += blockDim.x) mx = fmaxf(mx, fmaxf(fabsf(row[i].x), fabsf(row[i].y)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) mx = fmaxf(mx, red[w]);
+  int e = (int)((__float_as_uint(mx) >> 23) & 0xff);    // mx < 2^(e - 126)
+  e = e < 15 ? 15 : (e > 254 ? 254 : e);
+  float f = __uint_as_float((unsigned)(268 - e) << 23);  // 2^(141 - e): mx f < 2^15
+  float inv = __uint_as_float((unsigned)(e - 14) << 23); // 2^(e - 141)
+  if (mx == 0.f) { f = 1.f; inv = 1.f; }
+  for (int i = tid; i < M; i += blockDim.x)
+    out[(size_t)c * M + i] = __floats2half2_rn(row[i].x * f, row[i].y * f);
+  if (tid == 0) inv_scale[c] = inv;
+}
+
+cudaError_t launch_spectrum_to_f16(const float2* spec, unsigned char* out, int D, const Layout& y, cudaStream_t s) {
+  spectrum_to_f16_kernel<<<D, 256, 0, s>>>(spec, reinterpret_cast<__half2*>(out),
+                                           reinterpret_cast<float*>(out + spec16_scales_offset_bytes(y, D)), y.M);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the table region is copied as it is
+  return cudaMemcpyAsync(out + spec16_tables_offset_bytes(y, D), spec + tables_offset(y, D),
+                         sizeof(float2) * (size_t)y.table_len, cudaMemcpyDeviceToDevice, s);
 }
 
 }  // namespace hyena

@@ -168,6 +168,52 @@ hyena_status hyena_forward_static_workspace(const void *v, const void *const *x,
                                             int D, int L, int N, hyena_dtype dtype, void *y, hyena_stream stream);
 
 /*
+ * Reduced-precision filter spectra (no counterpart on the pages, which fix
+ * no precision for the cached spectrum: page "Hyena Hierarchy ... long
+ * convolution language models", section 計算方法, only states that the long
+ * convolution runs through the FFT). The forward reads the spectrum of every
+ * filter once per channel, and at D*L of that size the float32 spectrum is
+ * the largest stream of a step; the f16 block halves it.
+ *
+ * Block of hyena_filter_spectrum_bytes_f16(D, L) bytes (0 when L is
+ * unsupported or D < 1):
+ *   [0, 4*D*M)            bins of the float32 block, same library order, as
+ *                         f16 pairs (re, im) scaled by s_c
+ *   [4*D*M, 4*D*M + 4*D)  1/s_c per channel, float32
+ *   (rounded up to 16 bytes) the float32 block's FFT tables, copied
+ * s_c is the power of two that brings every component of channel c below
+ * 2^15 in magnitude (1 for an all-zero channel), so scaling adds no error:
+ * each bin carries f16 rounding only (relative 2^-11 of the channel's
+ * largest component, or f16 subnormal spacing for bins more than 2^-24
+ * below it).
+ */
+size_t hyena_filter_spectrum_bytes_f16(int D, int L);
+
+/*
+ * hyena_filter_spectrum_to_f16 -- convert one float32 spectrum block
+ * (from hyena_filter_rfft, D channels, length L) into an f16 block.
+ *   hhat:   device, hyena_filter_spectrum_bytes(D, L) bytes, 16-byte aligned
+ *   hhat16: device, hyena_filter_spectrum_bytes_f16(D, L) bytes, 16-byte
+ *           aligned, must not overlap hhat
+ * Errors: HYENA_ERR_INVALID_ARG (alignment, D < 1), HYENA_ERR_UNSUPPORTED (L),
+ * HYENA_ERR_CUDA (launch). Asynchronous on stream.
+ */
+hyena_status hyena_filter_spectrum_to_f16(const void *hhat, int D, int L, void *hhat16, hyena_stream stream);
+
+/*
+ * hyena_forward_f16_spectra -- hyena_forward whose hhat[n] are f16 blocks
+ * from hyena_filter_spectrum_to_f16. Arguments, layouts, aliasing,
+ * workspace and errors are those of hyena_forward. It always runs the SIMT
+ * kernels (the tensor-core forward reads a float32 copy of its own). The
+ * result differs from hyena_forward by the f16 rounding of the spectra:
+ * relative L2 about 2^-11 per stage for spectra whose bins span a modest
+ * range.
+ */
+hyena_status hyena_forward_f16_spectra(const void *v, const void *const *x, const void *const *hhat16, int B, int D,
+                                       int L, int N, hyena_dtype dtype, void *y, void *workspace,
+                                       size_t workspace_bytes, hyena_stream stream);
+
+/*
  * Gradients (no counterpart printed on the pages, which only mention training
  * at 1M tokens: glossary "Hyena（ハイエナ）", section 超長系列タスクでの優位性). They are the chain
  * rule through the definitions above:

@@ -139,3 +139,26 @@ def test_striped_host_rejections(lib):
     assert lib.hyena_filter_exponential(p, p, 0, 3, 100, p, None) == hy.HYENA_ERR_INVALID_ARG
     assert lib.hyena_filter_exponential(p, p, 65, 3, 100, p, None) == hy.HYENA_ERR_INVALID_ARG
     del ok
+
+
+def test_f16_spectra_queries_and_host_rejections(lib):
+    p, mis = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    assert lib.hyena_filter_spectrum_bytes_f16(0, 1024) == 0
+    assert lib.hyena_filter_spectrum_bytes_f16(4, 1000) == 0
+    # bins, per-channel inverse scales (padded to 16 bytes), then the float32
+    # block's tables (a length without the tensor-core copy: bins, then tables)
+    M = 4096
+    f32 = lib.hyena_filter_spectrum_bytes(4, M)
+    tables = f32 - 8 * 4 * M
+    assert lib.hyena_filter_spectrum_bytes_f16(4, M) == 4 * 4 * M + 16 + tables
+    assert lib.hyena_filter_spectrum_to_f16(mis, 4, 1024, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_filter_spectrum_to_f16(p, 4, 1024, mis, None) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_filter_spectrum_to_f16(p, 0, 1024, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_filter_spectrum_to_f16(p, 4, 1000, p, None) == hy.HYENA_ERR_UNSUPPORTED
+    f = lib.hyena_forward_f16_spectra
+    xs = (ctypes.c_void_p * 2)(p, p)
+    assert f(p, xs, xs, 1, 1, 1024, 0, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1024, 2, 7, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(mis, xs, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1000, 2, 0, p, None, 0, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert f(p, xs, xs, 1, 1, 32768, 2, 0, p, None, 0, None) == hy.HYENA_ERR_WORKSPACE
