@@ -262,3 +262,47 @@ def exponential_filter(R, lam, L: int) -> np.ndarray:
     R, lam = _f64(np.atleast_2d(R)), _f64(np.atleast_2d(lam))
     t = np.arange(L, dtype=np.float64)
     return np.einsum("cn,cnt->ct", R, lam[:, :, None] ** t[None, None, :])
+
+
+# ------------------------------------------------------------------ HyenaND --
+# The N-dimensional operator of the HyenaND summary (page "HyenaND ... nSubQ",
+# section 手法: a global convolution evaluated on the L_1 x ... x L_N grid
+# itself through an N-dimensional FFT, with a circular boundary for periodic
+# systems or zero padding of the input to twice the grid for non-periodic
+# data). Plain numpy, float64; numpy's FFT is the only library step.
+
+def nd_conv(K, z, boundary: str) -> np.ndarray:
+    """ND convolution of z by the kernel K on one grid (both shaped dims).
+    circular:  y[p] = sum_q K[(p - q) mod dims] z[q]
+    zero:      y[p] = sum_{0 <= q <= p} K[p - q] z[q]   (linear convolution of
+               the grid signals, i.e. both zero-padded to 2 x dims; kept on the grid)"""
+    K, z = np.asarray(K, dtype=np.float64), np.asarray(z, dtype=np.float64)
+    assert K.shape == z.shape
+    dims = z.shape
+    if boundary == "circular":
+        return np.real(np.fft.ifftn(np.fft.fftn(K) * np.fft.fftn(z)))
+    if boundary != "zero":
+        raise ValueError(boundary)
+    s = tuple(2 * d for d in dims)
+    axes = tuple(range(len(dims)))
+    full = np.fft.irfftn(np.fft.rfftn(K, s, axes=axes) * np.fft.rfftn(z, s, axes=axes), s, axes=axes)
+    return full[tuple(slice(0, d) for d in dims)]
+
+
+def hyena_nd_forward(v, xs, Ks, dims, boundary: str, filter_row=None) -> np.ndarray:
+    """Order-N recurrence of the Hyena operator with the ND convolution:
+    z_1 = v, z_{n+1} = x_n . (K_n conv z_n), y = z_{N+1}, row by row.
+    v, xs[n]: [C][prod(dims)] (grid flattened row-major); Ks[n]: [F][prod(dims)];
+    filter_row[r] = the filter row of data row r (default r)."""
+    v = _f64(np.atleast_2d(v))
+    C = v.shape[0]
+    fr = np.arange(C) if filter_row is None else np.asarray(filter_row)
+    dims = tuple(int(d) for d in dims)
+    y = np.empty_like(v)
+    for r in range(C):
+        z = v[r].reshape(dims)
+        for n, x in enumerate(xs):
+            K = _f64(np.atleast_2d(Ks[n]))[fr[r]].reshape(dims)
+            z = _f64(np.atleast_2d(x))[r].reshape(dims) * nd_conv(K, z, boundary)
+        y[r] = z.reshape(-1)
+    return y
