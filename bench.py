@@ -22,6 +22,10 @@ and dh_n out.
 --pass striped times the StripedHyena-form operator q . (hG * (k . v)) with
 Hyena-SE filters (featurizers of 4 taps, inner filter of 7) on the workload's
 B, D, L: three inputs and one output of B*D*L elements each.
+--pass nd times the HyenaND forward (order-N recurrence with a 2-D or 3-D
+convolution, circular or zero-padded) on the ND workload --nd-config I; the
+metric counts B*D*grid points per second, the roofline v, x_n, y and the
+padded-grid spectra.
 """
 from __future__ import annotations
 
@@ -46,6 +50,8 @@ import synth  # noqa: E402
 METRIC = "Hyena order-N fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
 METRIC_BWD = "Hyena order-N bwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
 METRIC_STRIPED = "StripedHyena-SE fwd B·D·L/s (×1e9) and % of HBM roofline, 1 B200"
+METRIC_ND = "HyenaND order-N fwd B·D·grid/s (×1e9) and % of HBM roofline, 1 B200"
+UNIT_ND = "1e9 B*D*grid/s"
 STRIPED_LF, STRIPED_LG = 4, 7
 UNIT = "1e9 B*D*L/s"
 KERNEL_SOURCES = os.path.join(ROOT, "fft_long_convolution_implicit_b200", "csrc")
@@ -279,6 +285,176 @@ def oracle_striped_sample(w: synth.Workload, target_core_seconds: float = 8.0):
                       f"direct FIR sums", "seconds": dt}
 
 
+def oracle_nd_sample(w: "synth.NDWorkload", target_core_seconds: float = 8.0):
+    """The float64 HyenaND oracle (numpy FFT, one thread) on a bounded sample of rows."""
+    import oracle
+    K = synth.nd_kernels(w)
+
+    def run(rows):
+        v, xs = synth.nd_inputs(w, rows)
+        t0 = time.perf_counter()
+        oracle.hyena_nd_forward(v, xs, [K[n] for n in range(w.N)], w.dims, w.boundary,
+                                filter_row=[r % w.D for r in rows])
+        return time.perf_counter() - t0
+
+    per_row = max(run([0]), 1e-5)
+    nrows = int(min(w.channels, max(1, target_core_seconds / per_row)))
+    dt = run(list(range(nrows)))
+    return {"value": nrows * w.grid / dt / 1e9, "unit": UNIT_ND, "cores": 1, "kind": "oracle",
+            "sample": f"{nrows} of {w.channels} (b,c) rows of {w.name}, all N={w.N} stages, numpy FFT "
+                      f"({w.boundary} boundary)", "seconds": dt}
+
+
+def run_nd(args) -> int:
+    w = synth.nd_workload(args.nd_config)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = {"workload": w.name, "B": w.B, "D": w.D, "dims": list(w.dims), "boundary": w.boundary, "N": w.N,
+           "io": w.dtype, "pass": "nd"}
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = oracle_nd_sample(w)
+        print(json.dumps({"impl": "reference", "metric": METRIC_ND, "value": cb["value"], "unit": UNIT_ND,
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": w.channels * w.grid / (cb["value"] * 1e9) * 1e3, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+                          "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                          "e2e": {"value": cb["value"], "unit": UNIT_ND, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    import fft_long_convolution_implicit_b200 as hy
+    from fft_long_convolution_implicit_b200 import build as hybuild
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    else:
+        torch.cuda.set_device(0)
+    if rank == 0:
+        hybuild.build()
+    if world > 1:
+        dist.barrier()
+    hy.load()
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    wr = synth.NDWorkload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
+    v_np, xs_np = synth.nd_inputs(wr)
+    K = synth.nd_kernels(wr)
+    base_v = torch.from_numpy(v_np).view(w.B, w.D, w.grid).to(dev).to(dt)
+    base_x = [torch.from_numpy(x).view(w.B, w.D, w.grid).to(dev).to(dt) for x in xs_np]
+    base_k = [hy.nd_filter_spectrum(torch.from_numpy(K[n]).to(dev), w.dims, w.boundary) for n in range(w.N)]
+    set_bytes = (w.N + 2) * w.channels * w.grid * w.elem_bytes + sum(t.numel() for t in base_k)
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    sets = []
+    for i in range(nsets):
+        if i == 0:
+            v_s, x_s, k_s = base_v, base_x, base_k
+        else:
+            v_s, x_s, k_s = base_v.clone(), [x.clone() for x in base_x], [t.clone() for t in base_k]
+        sets.append(hy.PreparedND(v_s, x_s, k_s, w.dims, w.boundary, stream=stream))
+    torch.cuda.synchronize()
+    launches_per_step = count_kernel_nodes(lambda st: hy.PreparedND(base_v, base_x, base_k, w.dims, w.boundary,
+                                                                    stream=st))
+    for i in range(args.warmup):
+        sets[i % nsets]()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank if world > 1 else 0)
+    sampler.start()
+    time.sleep(0.2)
+    K_steps = args.steps
+    ev_pre = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    ev_post = [torch.cuda.Event(enable_timing=True) for _ in range(K_steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K_steps):
+        ev_pre[i].record(stream)
+        sets[i % nsets]()
+        ev_post[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dist if world > 1 else None, dev)
+    value = whole_job_throughput(K_steps * w.channels * w.grid, world, elapsed_ms)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev_pre, ev_post))
+    peak, peak_kind = hbm_peak()
+    alg_bytes = w.roofline_bytes()
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+
+    # end to end: pinned host inputs in, y out, through the same public call
+    pin_v = base_v.cpu().pin_memory()
+    pin_x = [x.cpu().pin_memory() for x in base_x]
+    dv = torch.empty_like(base_v)
+    dxs = [torch.empty_like(x) for x in base_x]
+    pin_y = torch.empty_like(pin_v).pin_memory()
+    e2e_call = hy.PreparedND(dv, dxs, base_k, w.dims, w.boundary, stream=stream)
+
+    def e2e_step():
+        dv.copy_(pin_v, non_blocking=True)
+        for d, p in zip(dxs, pin_x):
+            d.copy_(p, non_blocking=True)
+        pin_y.copy_(e2e_call(), non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    e2e_value = whole_job_throughput(args.e2e_steps * w.channels * w.grid, world, e2e_ms)
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC_ND, "value": round(value, 4), "unit": UNIT_ND, "n_gpus": world, "steps": K_steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {**cfg, "global_batch": w.B * world, "parallelism": f"replicas x{world}",
+                       "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
+                             f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "alg_bytes_per_launch": alg_bytes, "kernel": "nd_forward_kernel",
+                         "kernel_ms": round(kernel_ms, 5)},
+            "e2e": {"value": round(e2e_value, 4), "unit": UNIT_ND,
+                    "h2d_bytes_per_step": (w.N + 1) * w.channels * w.grid * w.elem_bytes,
+                    "d2h_bytes_per_step": w.channels * w.grid * w.elem_bytes, "ms_per_step": e2e_ms / args.e2e_steps},
+            "gpu_launches": K_steps * launches_per_step,
+            "clocks": clocks,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if not args.no_cpu_baseline and world == 1:
+            cb = oracle_nd_sample(w)
+            line["cpu_baseline"] = {k: round(cb[k], 6) if k == "value" else cb[k]
+                                    for k in ("value", "unit", "cores", "kind", "sample")}
+        elif not args.no_cpu_baseline:
+            line["cpu_baseline"] = None
+        print(json.dumps(line))
+    return 0
+
+
 # ---------------------------------------------------------------- main --
 
 def main():
@@ -290,12 +466,17 @@ def main():
     ap.add_argument("--config", type=int, default=1, help="workload index (default 1: B=4 D=768 L=2048 N=2 bf16)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", choices=["forward", "backward", "striped"], default="forward")
+    ap.add_argument("--pass", dest="which", choices=["forward", "backward", "striped", "nd"], default="forward")
+    ap.add_argument("--nd-config", type=int, default=1, help="HyenaND workload index for --pass nd")
     ap.add_argument("--shape", default=None,
                     help="N,dtype,B,D,L: a custom shape instead of --config (small ncu captures)")
     ap.add_argument("--spectrum", choices=["f32", "f16"], default="f32",
                     help="forward pass: cached filter spectra as float32 (default) or f16 blocks")
     args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.which == "nd":
+        return run_nd(args)
     bwd = args.which == "backward"
     striped = args.which == "striped"
     metric = METRIC_BWD if bwd else (METRIC_STRIPED if striped else METRIC)

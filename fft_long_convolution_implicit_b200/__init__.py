@@ -31,6 +31,7 @@ EXPORTS = (
     "hyena_filter_backward_workspace_bytes", "hyena_filter_backward", "hyena_device_timeouts",
     "hyena_striped_forward", "hyena_striped_featurize", "hyena_filter_exponential",
     "hyena_filter_spectrum_bytes_f16", "hyena_filter_spectrum_to_f16", "hyena_forward_f16_spectra",
+    "hyena_nd_spectrum_bytes", "hyena_nd_filter_spectrum", "hyena_nd_forward",
 )
 
 
@@ -82,6 +83,12 @@ def load() -> ctypes.CDLL:
     l.hyena_filter_spectrum_to_f16.restype = i
     l.hyena_forward_f16_spectra.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
     l.hyena_forward_f16_spectra.restype = i
+    l.hyena_nd_spectrum_bytes.argtypes = [i, i, ctypes.POINTER(i), i]
+    l.hyena_nd_spectrum_bytes.restype = sz
+    l.hyena_nd_filter_spectrum.argtypes = [P, i, i, ctypes.POINTER(i), i, P, P]
+    l.hyena_nd_filter_spectrum.restype = i
+    l.hyena_nd_forward.argtypes = [P, P, P, i, i, i, ctypes.POINTER(i), i, i, i, P, P]
+    l.hyena_nd_forward.restype = i
     l.hyena_forward_workspace_bytes.argtypes = [i, i, i, i, i]
     l.hyena_forward_workspace_bytes.restype = sz
     l.hyena_forward.argtypes = [P, P, P, i, i, i, i, i, P, P, sz, P]
@@ -369,6 +376,74 @@ def spectrum_natural(hhat, D: int, L: int):
     out[:, M] = blk[:, 0, 1].to(out.dtype)       # packed Nyquist bin
     out[:, 0] = blk[:, 0, 0].to(out.dtype)
     return out
+
+
+# ----------------------------------------------------------------- HyenaND --
+
+ND_BOUNDARY = {"zero": 0, "circular": 1}
+
+
+def _nd_dims(dims):
+    dims = tuple(int(d) for d in dims)
+    return dims, (ctypes.c_int * len(dims))(*dims)
+
+
+def nd_spectrum_bytes(D: int, dims, boundary: str) -> int:
+    dims, arr = _nd_dims(dims)
+    return load().hyena_nd_spectrum_bytes(D, len(dims), arr, ND_BOUNDARY[boundary])
+
+
+def nd_filter_spectrum(K, dims, boundary: str, khat=None, stream=None):
+    """Spectrum block (uint8 CUDA tensor) of one HyenaND kernel K: float32
+    [D][grid] (or [D][*dims]) on the grid dims, boundary "zero" or "circular"."""
+    torch = _torch()
+    dims, arr = _nd_dims(dims)
+    D = K.shape[0]
+    nbytes = nd_spectrum_bytes(D, dims, boundary)
+    if nbytes == 0:
+        _check(HYENA_ERR_UNSUPPORTED, "hyena_nd_spectrum_bytes")
+    if khat is None:
+        khat = torch.empty(nbytes, dtype=torch.uint8, device=K.device)
+    _check(load().hyena_nd_filter_spectrum(_dev(K, "K"), D, len(dims), arr, ND_BOUNDARY[boundary], _dev(khat, "khat"),
+                                           _stream(stream)), "hyena_nd_filter_spectrum")
+    return khat
+
+
+class PreparedND:
+    """hyena_nd_forward with its arguments marshalled once: v and xs are
+    [B][D][grid] (or [B][D][*dims]) float32 or bfloat16, khats from
+    nd_filter_spectrum; calling it issues the C call only."""
+
+    def __init__(self, v, xs, khats, dims, boundary: str, y=None, stream=None):
+        torch = _torch()
+        B, D = v.shape[0], v.shape[1]
+        N = len(xs)
+        if len(khats) != N:
+            raise ValueError("need one spectrum per gate")
+        code = _dtype_code(v)
+        for x in xs:
+            if x.shape != v.shape or x.dtype != v.dtype:
+                raise ValueError("gates must match v in shape and dtype")
+        self.y = torch.empty_like(v) if y is None else y
+        self.dims, self._dims = _nd_dims(dims)
+        self._keep = (v, list(xs), list(khats))
+        self._x = (ctypes.c_void_p * N)(*[_dev(x, "x").value for x in xs])
+        self._h = (ctypes.c_void_p * N)(*[_dev(h, "khat").value for h in khats])
+        self._args = (_dev(v, "v"), self._x, self._h, B, D, len(self.dims), self._dims, ND_BOUNDARY[boundary], N, code,
+                      _dev(self.y, "y"), _stream(stream))
+        self._fn = load().hyena_nd_forward
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != HYENA_OK:
+            raise HyenaError(st, "hyena_nd_forward")
+        return self.y
+
+
+def nd_forward(v, xs, khats, dims, boundary: str, y=None, stream=None):
+    """HyenaND order-N forward: y = z_{N+1} with z_{n+1} = x_n . (K_n conv z_n)
+    on the grid dims (boundary "zero" or "circular")."""
+    return PreparedND(v, xs, khats, dims, boundary, y=y, stream=stream)()
 
 
 class PreparedForward:

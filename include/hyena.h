@@ -326,6 +326,55 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
  */
 hyena_status hyena_device_timeouts(void);
 
+/*
+ * HyenaND (HyenaND summary, section 手法: a global convolution evaluated on
+ * the L_1 x ... x L_nd grid through an nd-dimensional FFT; circular for
+ * periodic data, or with the input zero-padded to twice the grid so that
+ * nothing leaks across the boundary). The order-N recurrence of
+ * hyena_forward with the causal 1-D sum replaced by
+ *   boundary HYENA_ND_CIRCULAR: (K conv z)[p] = sum_q K[(p - q) mod dims] z[q]
+ *   boundary HYENA_ND_ZERO:     (K conv z)[p] = sum_{0 <= q <= p} K[p - q] z[q]
+ *                               (componentwise q <= p: the linear convolution
+ *                               of the two grid signals, kept on the grid)
+ * K_n are given as values on the grid (offset 0 at index 0); how they are
+ * generated (the summary's SIREN/FiLM kernel and Gaussian window) is up to
+ * the caller.
+ *
+ * Shapes: nd in 1..3, dims[a] powers of two (host array of nd ints, row-major
+ * grid, axis nd-1 contiguous); padded axis P_a = 2 dims[a] (zero) or dims[a]
+ * (circular) at most 1024, and P = prod P_a at most 16384. Others return
+ * HYENA_ERR_UNSUPPORTED (0 bytes from hyena_nd_spectrum_bytes).
+ */
+#define HYENA_ND_ZERO 0
+#define HYENA_ND_CIRCULAR 1
+
+/* Bytes of one filter's spectrum block: [D][P] float2 then a twiddle table. */
+size_t hyena_nd_spectrum_bytes(int D, int nd, const int *dims, int boundary);
+
+/*
+ * hyena_nd_filter_spectrum -- cache the spectrum of ONE filter:
+ *   K:    device float32 [D][grid] (16-byte aligned)
+ *   khat: device block of hyena_nd_spectrum_bytes(D, nd, dims, boundary)
+ *         bytes (16-byte aligned): the padded-grid DFT of K_c times 1/P in
+ *         the library's transform order (each axis index bit-reversed), then
+ *         the twiddle table the forward reads.
+ * Errors: HYENA_ERR_INVALID_ARG (pointers, D), HYENA_ERR_UNSUPPORTED (shape),
+ * HYENA_ERR_CUDA (launch). Asynchronous on stream.
+ */
+hyena_status hyena_nd_filter_spectrum(const float *K, int D, int nd, const int *dims, int boundary, void *khat,
+                                      hyena_stream stream);
+
+/*
+ * hyena_nd_forward -- y = z_{N+1} of the recurrence above.
+ *   v, x[n], y: device [B][D][grid] in dtype (16-byte aligned); x is a host
+ *         array of N device pointers; y may alias v or any x[n]
+ *   khat: host array of N device pointers to blocks from
+ *         hyena_nd_filter_spectrum (same D, nd, dims, boundary)
+ * No workspace: every stage stays on chip. Errors as hyena_forward.
+ */
+hyena_status hyena_nd_forward(const void *v, const void *const *x, const void *const *khat, int B, int D, int nd,
+                              const int *dims, int boundary, int N, hyena_dtype dtype, void *y, hyena_stream stream);
+
 /* HYENA_ABI_VERSION of the loaded library. */
 int hyena_abi_version(void);
 

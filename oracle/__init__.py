@@ -298,11 +298,13 @@ def hyena_nd_forward(v, xs, Ks, dims, boundary: str, filter_row=None) -> np.ndar
     C = v.shape[0]
     fr = np.arange(C) if filter_row is None else np.asarray(filter_row)
     dims = tuple(int(d) for d in dims)
+    Ks = [np.atleast_2d(k) for k in Ks]
+    xs = [np.atleast_2d(x) for x in xs]
     y = np.empty_like(v)
     for r in range(C):
         z = v[r].reshape(dims)
         for n, x in enumerate(xs):
-            K = _f64(np.atleast_2d(Ks[n]))[fr[r]].reshape(dims)
-            z = _f64(np.atleast_2d(x))[r].reshape(dims) * nd_conv(K, z, boundary)
+            K = _f64(Ks[n][fr[r]]).reshape(dims)
+            z = _f64(x[r]).reshape(dims) * nd_conv(K, z, boundary)
         y[r] = z.reshape(-1)
     return y

@@ -278,3 +278,95 @@ def sample_rows(w: Workload, count: int, salt: int = 0) -> list[int]:
             break
         picks.add(int(val % np.uint64(C)))
     return sorted(picks)
+
+
+# --------------------------------------------------------------------------
+# HyenaND workloads: the order-N recurrence on a 2-D or 3-D grid. Inputs use
+# the 1-D generators on the flattened grid (row-major, last axis contiguous);
+# kernels K_n are N(0,1) values under a Gaussian window (the summary's kernel
+# carries a learnable Gaussian window), one width per channel.
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class NDWorkload:
+    name: str
+    N: int
+    dtype: str
+    B: int
+    D: int
+    dims: tuple
+    boundary: str          # "zero" or "circular"
+    gamma_lo: float = 2.0
+    gamma_hi: float = 32.0
+    seed: int = 1100
+
+    @property
+    def grid(self) -> int:
+        return int(np.prod(self.dims))
+
+    @property
+    def padded(self) -> int:
+        return int(np.prod([2 * d if self.boundary == "zero" else d for d in self.dims]))
+
+    @property
+    def channels(self) -> int:
+        return self.B * self.D
+
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    def flat(self) -> Workload:
+        return Workload(self.name, self.N, self.dtype, self.B, self.D, self.grid, 0.5, 20.0, seed=self.seed)
+
+    def roofline_bytes(self) -> int:
+        """(N+2) B D grid elem (v, x_n, y) + N D P complex64 (the cached padded-grid
+        spectra), each touched once."""
+        return (self.N + 2) * self.B * self.D * self.grid * self.elem_bytes + self.N * self.D * self.padded * 8
+
+
+ND_WORKLOADS = [
+    NDWorkload("hyenand2_f32_B3_D4_8x16_zero", 2, "f32", 3, 4, (8, 16), "zero", seed=1100),
+    NDWorkload("hyenand2_bf16_B2_D256_64x64_zero", 2, "bf16", 2, 256, (64, 64), "zero", seed=1101),
+    NDWorkload("hyenand2_bf16_B2_D256_128x128_circular", 2, "bf16", 2, 256, (128, 128), "circular", seed=1102),
+    NDWorkload("hyenand2_bf16_B2_D256_8x16x16_zero", 2, "bf16", 2, 256, (8, 16, 16), "zero", seed=1103),
+    NDWorkload("hyenand2_bf16_B2_D256_16x32x32_circular", 2, "bf16", 2, 256, (16, 32, 32), "circular", seed=1104),
+]
+
+
+def nd_workload(i: int) -> NDWorkload:
+    return ND_WORKLOADS[i]
+
+
+def nd_custom(N: int, dtype: str, B: int, D: int, dims, boundary: str, seed: int = 17) -> NDWorkload:
+    dims = tuple(int(d) for d in dims)
+    return NDWorkload(f"custom_nd_N{N}_{dtype}_B{B}_D{D}_{'x'.join(map(str, dims))}_{boundary}", N, dtype, B, D,
+                      dims, boundary, seed=seed)
+
+
+def nd_inputs(w: NDWorkload, rows: list[int] | None = None):
+    """(v, [x_1..x_N]) as float32 [len(rows)][grid] (storage-rounded)."""
+    return inputs(w.flat(), rows)
+
+
+def nd_kernels(w: NDWorkload) -> np.ndarray:
+    """K float32 [N][D][grid]: N(0,1) times exp(-gamma_c sum_a (d_a / L_a)^2),
+    d_a the offset along axis a (circular: the periodic distance), gamma_c
+    geometric from gamma_lo to gamma_hi over the channels; each kernel scaled
+    to unit L2 norm of its window."""
+    coords = np.meshgrid(*[np.arange(d, dtype=np.float64) for d in w.dims], indexing="ij")
+    r2 = np.zeros(w.dims)
+    for a, d in enumerate(w.dims):
+        off = coords[a]
+        if w.boundary == "circular":
+            off = np.minimum(off, d - off)
+        r2 += (off / d) ** 2
+    r2 = r2.reshape(-1)
+    K = np.empty((w.N, w.D, w.grid), dtype=np.float32)
+    for c in range(w.D):
+        gamma = w.gamma_lo * (w.gamma_hi / w.gamma_lo) ** (c / max(1, w.D - 1))
+        win = np.exp(-gamma * r2)
+        win /= np.linalg.norm(win)
+        for n in range(w.N):
+            K[n, c] = normal(w.seed, 500 + n, c * w.grid, w.grid) * win
+    return K

@@ -162,3 +162,31 @@ def test_f16_spectra_queries_and_host_rejections(lib):
     assert f(mis, xs, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
     assert f(p, xs, xs, 1, 1, 1000, 2, 0, p, None, 0, None) == hy.HYENA_ERR_UNSUPPORTED
     assert f(p, xs, xs, 1, 1, 32768, 2, 0, p, None, 0, None) == hy.HYENA_ERR_WORKSPACE
+
+
+def test_nd_queries_and_host_rejections(lib):
+    p, mis = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    I3 = ctypes.c_int * 3
+    # [D][P] float2 then the twiddle table (half the longest padded axis, even count)
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(64, 64, 0), 0) == 8 * (4 * 128 * 128 + 64)
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(128, 128, 0), 1) == 8 * (4 * 128 * 128 + 64)
+    assert lib.hyena_nd_spectrum_bytes(1, 3, I3(2, 2, 2), 1) == 8 * (8 + 2)
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(128, 128, 0), 0) == 0      # padded grid above 16384 points
+    assert lib.hyena_nd_spectrum_bytes(4, 1, I3(1024, 0, 0), 0) == 0       # padded axis above 1024
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(12, 16, 0), 0) == 0        # not a power of two
+    assert lib.hyena_nd_spectrum_bytes(4, 4, I3(2, 2, 2), 0) == 0          # nd above 3
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(8, 8, 0), 2) == 0          # unknown boundary
+    assert lib.hyena_nd_spectrum_bytes(0, 2, I3(8, 8, 0), 0) == 0
+    f = lib.hyena_nd_filter_spectrum
+    assert f(mis, 4, 2, I3(8, 8, 0), 0, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, 4, 2, I3(8, 8, 0), 0, mis, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, 4, 2, I3(12, 8, 0), 0, p, None) == hy.HYENA_ERR_UNSUPPORTED
+    g = lib.hyena_nd_forward
+    xs = (ctypes.c_void_p * 2)(p, p)
+    ok = I3(8, 8, 0)
+    assert g(p, xs, xs, 1, 1, 2, ok, 0, 0, 0, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert g(p, xs, xs, 1, 1, 2, ok, 0, 2, 7, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert g(mis, xs, xs, 1, 1, 2, ok, 0, 2, 0, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert g(p, xs, xs, 0, 1, 2, ok, 0, 2, 0, p, None) == hy.HYENA_ERR_INVALID_ARG
+    assert g(p, xs, xs, 1, 1, 2, I3(8, 6, 0), 0, 2, 0, p, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert g(p, xs, xs, 1, 1, 0, ok, 0, 2, 0, p, None) == hy.HYENA_ERR_UNSUPPORTED
