@@ -12,12 +12,17 @@
 // pair are the real and imaginary parts of one complex grid (K is real, so one
 // complex convolution carries both), held in shared memory on the padded grid
 // P_1 x ... x P_nd (P_a = 2 L_a zero-padded, L_a circular; P = prod P_a <=
-// 16384 points, 128 KB). The transform is separable: along every axis,
-// in-place decimation-in-frequency radix-4 levels (one radix-2 level first
-// when log2 P_a is odd) leave each axis index bit-reversed; the spectrum
-// block K^ is stored in that same order, so the product needs no reordering,
-// and the inverse runs the levels backwards (decimation in time, conjugate
-// twiddles), returning natural order. K^ carries the 1/P of the inverse.
+// 16384 points, 128 KB plus one spare slot per 16 points against bank
+// conflicts). The transform is separable: along every axis, in-place
+// decimation-in-frequency steps of radix 2^k (k <= 4, DFT_R in registers,
+// then the twiddles w_m^{j r}, output r stored at the bit-reversed slot)
+// leave each axis index bit-reversed, exactly as 2-point levels would; the
+// spectrum block K^ is stored in that order, so the product needs no
+// reordering, and the inverse undoes the steps in reverse (decimation in
+// time, conjugate twiddles), returning natural order. K^ carries the 1/P of
+// the inverse. Register-resident fusions: the last forward step, the product
+// and the first inverse step share one pass; the last inverse step, the gate
+// x_n and the next stage's first forward step (same positions) share another.
 // All N stages stay in shared memory; only v, x_n and y touch HBM, plus K^.
 #include <cuda_bf16.h>
 
@@ -32,15 +37,21 @@ constexpr int kNdMaxDims = 3;
 constexpr int kNdMaxLogP = 14;      // 16384 complex points: 128 KB of shared memory
 constexpr int kNdMaxLogAxis = 10;   // padded axis length <= 1024 (twiddle table <= 512 entries)
 
+constexpr int kNdMaxSteps = 9;      // <= 3 radix steps per axis (padded axis <= 2^10)
+
 struct NdGeom {
   int nd;
   int logP;
   int logn[kNdMaxDims];   // padded axis lengths
   int logs[kNdMaxDims];   // inner stride of each axis on the padded grid
   int logL[kNdMaxDims];   // grid axis lengths
-  int logT;               // table length 2^(logT - 1): w_T^k for k < T/2, T = longest padded axis
+  int logT;               // twiddle table w_T^k, k < T, T = longest padded axis (at least 2)
   int G;                  // grid points prod L_a
   int zero;               // zero-padded boundary
+  // forward radix steps, axis 0 first; step i works along axis st_a[i] on
+  // blocks of 2^st_logm[i] points with radix 2^st_logR[i]
+  int nsteps;
+  signed char st_a[kNdMaxSteps], st_logm[kNdMaxSteps], st_logR[kNdMaxSteps];
 };
 
 __device__ __forceinline__ float ld1(const float* p) { return __ldg(p); }
@@ -80,6 +91,8 @@ __device__ __forceinline__ int pos_to_grid(const NdGeom& g, int pos) {
   return gi;
 }
 
+// Spectrum kernel transform: 2-point levels, two at a time (same output order
+// as the radix steps of the forward kernel).
 // One radix-2 level (block size 2^logm) along an axis of inner stride 2^logs.
 template <bool INV>
 __device__ __forceinline__ void level2(float2* s, const float2* tw, int logT, int logm, int logs, int P, int tid,
@@ -175,65 +188,364 @@ struct NdGates {
   const T* p[kMaxOrder];
 };
 
+// Shared-memory slot of padded-grid position pos: one spare slot after every
+// 16 points keeps the radix steps along the contiguous axis free of bank
+// conflicts.
+__device__ __forceinline__ int spad(int pos) { return pos + (pos >> 4); }
+
+__host__ __device__ constexpr int brev_bits(int r, int bits) {
+  int o = 0;
+  for (int i = 0; i < bits; ++i) o |= ((r >> i) & 1) << (bits - 1 - i);
+  return o;
+}
+
+template <int R>
+constexpr int log2_of() {
+  return R == 2 ? 1 : R == 4 ? 2 : R == 8 ? 3 : 4;
+}
+
+// Step i: blocks of 2^logm points, 2^logq butterflies per block, along an
+// axis of inner stride 2^logs (read once per pass from the shared geometry).
+struct StepGeo {
+  int logs, logq, logm;
+};
+__device__ __forceinline__ StepGeo step_geo(const NdGeom& g, int i) {
+  StepGeo q;
+  q.logm = g.st_logm[i];
+  q.logq = q.logm - g.st_logR[i];
+  q.logs = g.logs[g.st_a[i]];
+  return q;
+}
+
+// Butterfly t: positions base + r * stride (r < R) in the padded grid;
+// in = offset along the inner axes, j = offset inside its block.
+struct StepIdx {
+  int base, stride, j, logm, in;
+};
+__device__ __forceinline__ StepIdx step_index(const StepGeo& q, int t) {
+  const int in = t & ((1 << q.logs) - 1);
+  const int r = t >> q.logs;
+  const int j = r & ((1 << q.logq) - 1);
+  const int blk = r >> q.logq;
+  return {(((blk << q.logm) + j) << q.logs) + in, 1 << (q.logq + q.logs), j, q.logm, in};
+}
+
+// Grid index of the inner-axes offset `in` of a step along axis 0 (the
+// flattened axes 1 .. nd-1 of the padded grid), or -1 in the padding.
+__device__ __forceinline__ int inner_to_grid(const NdGeom& g, int in) {
+  int gi = 0;
+#pragma unroll
+  for (int a = 1; a < kNdMaxDims; ++a) {
+    if (a < g.nd) {
+      const int coord = (in >> g.logs[a]) & ((1 << g.logn[a]) - 1);
+      if (coord >> g.logL[a]) return -1;
+      gi = (gi << g.logL[a]) + coord;
+    }
+  }
+  return gi;
+}
+
+// a[r] *= w_m^{j r} (forward) or its conjugate (inverse); w_m^k = tw[k T / m].
+// Powers come from w^j (and w^{8j}) by at most three products.
+template <int R, bool INV>
+__device__ __forceinline__ void step_twiddle(float2 (&a)[R], const float2* tw, int logT, int logm, int j) {
+  const int sh = logT - logm;
+  float2 w[R];
+  w[0] = make_float2(1.f, 0.f);
+  w[1] = tw[j << sh];
+  if constexpr (R >= 4) {
+    w[2] = cmul(w[1], w[1]);
+    w[3] = cmul(w[2], w[1]);
+  }
+  if constexpr (R >= 8) {
+    w[4] = cmul(w[2], w[2]);
+    w[5] = cmul(w[4], w[1]);
+    w[6] = cmul(w[4], w[2]);
+    w[7] = cmul(w[4], w[3]);
+  }
+  if constexpr (R >= 16) {
+    w[8] = tw[(8 * j) << sh];
+#pragma unroll
+    for (int r = 9; r < 16; ++r) w[r] = cmul(w[8], w[r - 8]);
+  }
+#pragma unroll
+  for (int r = 1; r < R; ++r) a[r] = INV ? cmulc(a[r], w[r]) : cmul(a[r], w[r]);
+}
+
+// Decimation-in-frequency step: a (natural order over r) -> DFT_R, twiddles;
+// output r belongs at position base + bitrev(r) * stride.
+template <int R>
+__device__ __forceinline__ void dif(float2 (&a)[R], const float2* tw, int logT, const StepIdx& x) {
+  dftR<R, false, 0>(a);
+  step_twiddle<R, false>(a, tw, logT, x.logm, x.j);
+}
+// Its inverse (times R): a[r] from position base + bitrev(r) * stride ->
+// natural order over r.
+template <int R>
+__device__ __forceinline__ void dit(float2 (&a)[R], const float2* tw, int logT, const StepIdx& x) {
+  step_twiddle<R, true>(a, tw, logT, x.logm, x.j);
+  dftR<R, true, 0>(a);
+}
+
+template <int R, bool INV>
+__device__ void plain_step(float2* s, const float2* tw, const NdGeom& g, int i, int tid, int nt) {
+  constexpr int LR = log2_of<R>();
+  const StepGeo q = step_geo(g, i);
+  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  for (int t = tid; t < nb; t += nt) {
+    const StepIdx x = step_index(q, t);
+    float2 a[R];
+    if (!INV) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + r * x.stride)];
+      dif<R>(a, tw, logT, x);
+#pragma unroll
+      for (int r = 0; r < R; ++r) s[spad(x.base + brev_bits(r, LR) * x.stride)] = a[r];
+    } else {
+#pragma unroll
+      for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + brev_bits(r, LR) * x.stride)];
+      dit<R>(a, tw, logT, x);
+#pragma unroll
+      for (int r = 0; r < R; ++r) s[spad(x.base + r * x.stride)] = a[r];
+    }
+  }
+}
+
+// The last forward step, the product with the spectrum and the first inverse
+// step in registers (the two steps cover the same positions). The last step
+// runs along the innermost axis with one butterfly per block, so its R points
+// are contiguous (stride 1): their spectrum values are fetched first, as
+// 16-byte loads, to overlap the forward DFT.
+template <int R>
+__device__ void turn_step(float2* s, const float2* tw, const NdGeom& g, int i, const float2* __restrict__ H, int tid,
+                          int nt) {
+  constexpr int LR = log2_of<R>();
+  const StepGeo q = step_geo(g, i);
+  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  for (int t = tid; t < nb; t += nt) {
+    const StepIdx x = step_index(q, t);
+    float2 hk[R];
+    const float4* __restrict__ h4 = reinterpret_cast<const float4*>(H + x.base);
+#pragma unroll
+    for (int k = 0; k < R / 2; ++k) {
+      const float4 u = __ldg(h4 + k);
+      hk[2 * k] = make_float2(u.x, u.y);
+      hk[2 * k + 1] = make_float2(u.z, u.w);
+    }
+    float2 a[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + r)];
+    dif<R>(a, tw, logT, x);
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r] = cmul(a[r], hk[brev_bits(r, LR)]);
+    dit<R>(a, tw, logT, x);
+#pragma unroll
+    for (int r = 0; r < R; ++r) s[spad(x.base + r)] = a[r];
+  }
+}
+
+// Gate (or v) values of the pair's two rows: from shared-memory copies made
+// with cp.async while earlier passes ran, or straight from global memory.
+template <typename T, bool STAGED>
+struct PairSrc {
+  const T* r0;
+  const T* r1;
+  bool has1;
+  __device__ __forceinline__ float2 at(int gi) const {
+    if constexpr (STAGED) {
+      return make_float2(to_f(r0[gi]), has1 ? to_f(r1[gi]) : 0.f);
+    } else {
+      return make_float2(ld1(r0 + gi), has1 ? ld1(r1 + gi) : 0.f);
+    }
+  }
+  static __device__ __forceinline__ float to_f(float v) { return v; }
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+};
+
+// Steps 0 run along axis 0 over whole axes (one block), so butterfly t holds
+// axis-0 coordinates j + r q at the inner offset in: the grid index is
+// (j + r q) * (G / L_0) + inner_to_grid(in) inside the grid.
+struct Axis0Map {
+  int gin;        // grid index of the inner offset, -1 in the padding
+  int gstride;    // G / L_0
+  int L0;
+};
+
+// First forward step of stage 1 straight from v.
+template <int R, typename T, bool STAGED>
+__device__ void entry_step(float2* s, const float2* tw, const NdGeom& g, PairSrc<T, STAGED> src, int tid, int nt) {
+  constexpr int LR = log2_of<R>();
+  const StepGeo q = step_geo(g, 0);
+  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  const int L0 = 1 << g.logL[0], gstride = g.G >> g.logL[0], qn = 1 << q.logq;
+  for (int t = tid; t < nb; t += nt) {
+    const StepIdx x = step_index(q, t);
+    const int gin = inner_to_grid(g, x.in);
+    float2 a[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int c0 = x.j + r * qn;
+      a[r] = (gin < 0 || c0 >= L0) ? make_float2(0.f, 0.f) : src.at(c0 * gstride + gin);
+    }
+    dif<R>(a, tw, logT, x);
+#pragma unroll
+    for (int r = 0; r < R; ++r) s[spad(x.base + brev_bits(r, LR) * x.stride)] = a[r];
+  }
+}
+
+// Last inverse step of a stage, the gate x_n, then either the next stage's
+// first forward step (same positions) or the store of y.
+template <int R, bool LAST, typename T, bool STAGED>
+__device__ void exit_step(float2* s, const float2* tw, const NdGeom& g, PairSrc<T, STAGED> xg, T* __restrict__ y,
+                          size_t row0, size_t row1, int tid, int nt) {
+  constexpr int LR = log2_of<R>();
+  const StepGeo q = step_geo(g, 0);
+  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  const int L0 = 1 << g.logL[0], gstride = g.G >> g.logL[0], qn = 1 << q.logq;
+  for (int t = tid; t < nb; t += nt) {
+    const StepIdx x = step_index(q, t);
+    const int gin = inner_to_grid(g, x.in);
+    float2 a[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + brev_bits(r, LR) * x.stride)];
+    dit<R>(a, tw, logT, x);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int c0 = x.j + r * qn;
+      if (gin < 0 || c0 >= L0) {
+        a[r] = make_float2(0.f, 0.f);
+      } else {
+        const int gi = c0 * gstride + gin;
+        const float2 xv = xg.at(gi);
+        a[r] = make_float2(a[r].x * xv.x, a[r].y * xv.y);
+        if (LAST) {
+          st1(y + row0 + gi, a[r].x);
+          if (xg.has1) st1(y + row1 + gi, a[r].y);
+        }
+      }
+    }
+    if (!LAST) {
+      dif<R>(a, tw, logT, x);
+#pragma unroll
+      for (int r = 0; r < R; ++r) s[spad(x.base + brev_bits(r, LR) * x.stride)] = a[r];
+    }
+  }
+}
+
+#define ND_RADIX_SWITCH(LOGR, CALL) \
+  switch (LOGR) {                   \
+    case 1: { constexpr int R = 2; CALL; } break;  \
+    case 2: { constexpr int R = 4; CALL; } break;  \
+    case 3: { constexpr int R = 8; CALL; } break;  \
+    default: { constexpr int R = 16; CALL; } break; \
+  }
+
+// Copy the pair's two rows (G elements each) into shared memory with cp.async
+// (16-byte pieces; rows are 16-byte aligned when staging is enabled).
 template <typename T>
-__global__ void __launch_bounds__(1024) nd_forward_kernel(const T* __restrict__ v, NdGates<T> xs, SpecPtrs kh,
-                                                          T* __restrict__ y, NdGeom g, int B, int D, int N) {
+__device__ __forceinline__ void stage_rows(T* dst, const T* __restrict__ src, size_t row0, size_t row1, bool has1,
+                                           int G, int tid, int nt) {
+  const int nbytes = G * (int)sizeof(T);
+  block_copy_async(dst, src + row0, nbytes, tid, nt);
+  if (has1) block_copy_async(dst + G, src + row1, nbytes, tid, nt);
+  cp_async_commit();
+}
+
+template <typename T, bool STAGED>
+__global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v, NdGates<T> xs, SpecPtrs kh,
+                                                         T* __restrict__ y, NdGeom gp, int B, int D, int N) {
+  // the step tables are indexed at run time: read them from shared memory
+  __shared__ NdGeom g;
+  if (threadIdx.x == 0) g = gp;
   extern __shared__ float4 nd_smem_raw[];
   float2* s = reinterpret_cast<float2*>(nd_smem_raw);
-  const int P = 1 << g.logP;
-  float2* tw = s + P;
+  const int P = 1 << gp.logP;
+  float2* tw = s + spad(P) + 1;
+  // staged rows (STAGED): [2][G] elements after the table, 16-byte aligned
+  T* xb = reinterpret_cast<T*>(reinterpret_cast<char*>(nd_smem_raw) +
+                               ((sizeof(float2) * ((size_t)spad(P) + 1 + ((size_t)1 << gp.logT)) + 15) & ~(size_t)15));
   const int tid = threadIdx.x, nt = blockDim.x;
   const int c = blockIdx.x % D;
   const int b0 = 2 * (blockIdx.x / D);
+  const int G = gp.G;
+  const size_t row0 = ((size_t)b0 * D + c) * (size_t)G;
+  const size_t row1 = row0 + (size_t)D * (size_t)G;
   const bool has1 = b0 + 1 < B;
-  const size_t G = (size_t)g.G;
-  const size_t row0 = ((size_t)b0 * D + c) * G;
-  const size_t row1 = row0 + (size_t)D * G;
+  const int F = gp.nsteps;
 
+  if (STAGED) stage_rows(xb, v, row0, row1, has1, G, tid, nt);
   const float2* tsrc = kh.p[0] + (size_t)D * P;
-  for (int i = tid; i < (1 << (g.logT - 1)); i += nt) tw[i] = __ldg(tsrc + i);
-  if (g.zero)
-    for (int i = tid; i < P; i += nt) s[i] = make_float2(0.f, 0.f);
+  for (int i = tid; i < (1 << gp.logT); i += nt) tw[i] = __ldg(tsrc + i);
+  if (STAGED) cp_async_wait_all();
   __syncthreads();
-  for (int gi = tid; gi < g.G; gi += nt)
-    s[grid_to_pos(g, gi)] = make_float2(ld1(v + row0 + gi), has1 ? ld1(v + row1 + gi) : 0.f);
+
+  auto src_of = [&](const T* gsrc) {
+    PairSrc<T, STAGED> r;
+    r.r0 = STAGED ? xb : gsrc + row0;
+    r.r1 = STAGED ? xb + G : gsrc + row1;
+    r.has1 = has1;
+    return r;
+  };
+
+  if (F >= 2) {
+    ND_RADIX_SWITCH(g.st_logR[0], (entry_step<R, T, STAGED>(s, tw, g, src_of(v), tid, nt)));
+  } else {
+    const PairSrc<T, STAGED> vs = src_of(v);
+    for (int i = tid; i < P; i += nt) {
+      const int gi = pos_to_grid(g, i);
+      s[spad(i)] = gi < 0 ? make_float2(0.f, 0.f) : vs.at(gi);
+    }
+  }
   __syncthreads();
 
   for (int n = 0; n < N; ++n) {
-    nd_transform<false>(s, tw, g, tid, nt);
     const float2* __restrict__ H = pick(kh, n) + (size_t)c * P;
-    for (int i = tid; i < P; i += nt) s[i] = cmul(s[i], __ldg(H + i));
-    __syncthreads();
-    nd_transform<true>(s, tw, g, tid, nt);
-    const T* __restrict__ x = pick(xs, n);
-    if (n + 1 < N) {
-      if (g.zero) {
-        for (int i = tid; i < P; i += nt) {
-          const int gi = pos_to_grid(g, i);
-          float2 z = make_float2(0.f, 0.f);
-          if (gi >= 0) {
-            const float2 u = s[i];
-            z = make_float2(u.x * ld1(x + row0 + gi), has1 ? u.y * ld1(x + row1 + gi) : 0.f);
-          }
-          s[i] = z;
-        }
-      } else {
-        for (int gi = tid; gi < g.G; gi += nt) {
-          const int i = grid_to_pos(g, gi);
-          const float2 u = s[i];
-          s[i] = make_float2(u.x * ld1(x + row0 + gi), has1 ? u.y * ld1(x + row1 + gi) : 0.f);
-        }
-      }
+    const T* __restrict__ x_n = pick(xs, n);
+    const bool last = n + 1 == N;
+    // the gate rows arrive while the transform runs
+    if (STAGED) stage_rows(xb, x_n, row0, row1, has1, G, tid, nt);
+    for (int i = 1; i + 1 < F; ++i) {
+      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, false>(s, tw, g, i, tid, nt)));
       __syncthreads();
+    }
+    if (F >= 1) {
+      ND_RADIX_SWITCH(g.st_logR[F - 1], (turn_step<R>(s, tw, g, F - 1, H, tid, nt)));
     } else {
-      for (int gi = tid; gi < g.G; gi += nt) {
-        const float2 u = s[grid_to_pos(g, gi)];
-        const float x0 = ld1(x + row0 + gi);
-        const float x1 = has1 ? ld1(x + row1 + gi) : 0.f;
-        st1(y + row0 + gi, u.x * x0);
-        if (has1) st1(y + row1 + gi, u.y * x1);
+      for (int i = tid; i < P; i += nt) s[spad(i)] = cmul(s[spad(i)], __ldg(H + i));
+    }
+    __syncthreads();
+    for (int i = F - 2; i >= 1; --i) {
+      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, true>(s, tw, g, i, tid, nt)));
+      __syncthreads();
+    }
+    if (STAGED) {
+      cp_async_wait_all();
+      __syncthreads();
+    }
+    const PairSrc<T, STAGED> xg = src_of(x_n);
+    if (F >= 2) {
+      if (last) {
+        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, true, T, STAGED>(s, tw, g, xg, y, row0, row1, tid, nt)));
+      } else {
+        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, false, T, STAGED>(s, tw, g, xg, y, row0, row1, tid, nt)));
+      }
+    } else {
+      for (int i = tid; i < P; i += nt) {
+        const int gi = pos_to_grid(g, i);
+        float2 u = make_float2(0.f, 0.f);
+        if (gi >= 0) {
+          const float2 a = s[spad(i)];
+          const float2 xv = xg.at(gi);
+          u = make_float2(a.x * xv.x, a.y * xv.y);
+          if (last) {
+            st1(y + row0 + gi, u.x);
+            if (has1) st1(y + row1 + gi, u.y);
+          }
+        }
+        s[spad(i)] = u;
       }
     }
+    __syncthreads();
   }
 }
 
@@ -261,10 +573,9 @@ __global__ void __launch_bounds__(1024) nd_spectrum_kernel(const float* __restri
   }
 }
 
-// w_T^k = exp(-2 pi i k / T), k < T/2, formed in double and rounded once.
+// w_T^k = exp(-2 pi i k / T), k < T, formed in double and rounded once.
 __global__ void nd_table_kernel(float2* __restrict__ tw, int logT) {
-  const int half = 1 << (logT - 1);
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < half; k += gridDim.x * blockDim.x) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < (1 << logT); k += gridDim.x * blockDim.x) {
     double sn, cs;
     sincospi(2.0 * (double)k / (double)(1 << logT), &sn, &cs);
     tw[k] = make_float2((float)cs, (float)-sn);
@@ -282,19 +593,25 @@ int ilog2_pow2(int x) {
 bool nd_geometry(int nd, const int* dims, int boundary, NdGeom* g) {
   if (nd < 1 || nd > kNdMaxDims || !dims || (boundary != 0 && boundary != 1)) return false;
   NdGeom r{};
-  r.nd = nd;
   r.zero = boundary == 0;
-  int logP = 0, logG = 0, logT = 1;
+  int logP = 0, logG = 0, logT = 1;   // the table has at least 2 entries
+  // axes of one point without padding change nothing and are dropped, so
+  // that step 0 always runs along the first kept axis
+  r.nd = 0;
   for (int a = 0; a < nd; ++a) {
     const int l = ilog2_pow2(dims[a]);
     if (l < 0) return false;
-    r.logL[a] = l;
-    r.logn[a] = l + (r.zero ? 1 : 0);
-    if (r.logn[a] > kNdMaxLogAxis) return false;
-    logP += r.logn[a];
+    const int ln = l + (r.zero ? 1 : 0);
+    if (ln > kNdMaxLogAxis) return false;
+    if (ln == 0) continue;
+    r.logL[r.nd] = l;
+    r.logn[r.nd] = ln;
+    ++r.nd;
+    logP += ln;
     logG += l;
-    if (r.logn[a] > logT) logT = r.logn[a];
+    if (ln > logT) logT = ln;
   }
+  nd = r.nd;
   if (logP > kNdMaxLogP) return false;
   int acc = 0;
   for (int a = nd - 1; a >= 0; --a) {
@@ -304,21 +621,56 @@ bool nd_geometry(int nd, const int* dims, int boundary, NdGeom* g) {
   r.logP = logP;
   r.logT = logT;
   r.G = 1 << logG;
+  // radix steps: ceil(log2 P_a / 4) per axis, the levels spread evenly
+  r.nsteps = 0;
+  for (int a = 0; a < nd; ++a) {
+    const int L = r.logn[a];
+    const int k = (L + 3) / 4;
+    int logm = L;
+    for (int q = 0; q < k; ++q) {
+      const int lr = L / k + (q < L % k ? 1 : 0);
+      r.st_a[r.nsteps] = (signed char)a;
+      r.st_logm[r.nsteps] = (signed char)logm;
+      r.st_logR[r.nsteps] = (signed char)lr;
+      ++r.nsteps;
+      logm -= lr;
+    }
+  }
+  // the spectral product runs on the last step, which must hold R contiguous
+  // points (one butterfly per block on an axis of inner stride 1)
+  if (r.nsteps > 0) {
+    const int l = r.nsteps - 1;
+    if (r.st_logm[l] != r.st_logR[l] || r.logs[r.st_a[l]] != 0) return false;
+  }
   *g = r;
   return true;
 }
 
 int nd_threads(const NdGeom& g) {
-  int t = (1 << g.logP) / 16;
+  int t = (1 << g.logP) / 32;
   if (t < 64) t = 64;
-  if (t > 1024) t = 1024;
+  if (t > 512) t = 512;
   return t;
 }
 
-size_t nd_smem(const NdGeom& g) { return sizeof(float2) * ((size_t)(1 << g.logP) + (1 << (g.logT - 1))); }
+// forward kernel: padded grid (+1 spare), the twiddle table, then (staged)
+// the pair's two rows of one input
+size_t nd_smem(const NdGeom& g, size_t elem, bool staged) {
+  const size_t P = (size_t)1 << g.logP;
+  const size_t base = (sizeof(float2) * (P + P / 16 + 1 + ((size_t)1 << g.logT)) + 15) & ~(size_t)15;
+  return base + (staged ? 2 * elem * (size_t)g.G : 0);
+}
+// staging wants 16-byte rows and room for them next to the grid
+bool nd_staged(const NdGeom& g, size_t elem) {
+  return (elem * (size_t)g.G) % 16 == 0 && nd_smem(g, elem, true) + sizeof(NdGeom) <= (size_t)227 * 1024;
+}
+// spectrum kernel: unpadded grid, then half the table
+size_t nd_spec_smem(const NdGeom& g) {
+  return sizeof(float2) * (((size_t)1 << g.logP) + ((size_t)1 << (g.logT - 1)));
+}
 
 size_t nd_block_bytes(const NdGeom& g, int D) {
-  return sizeof(float2) * ((size_t)D * (1 << g.logP) + (((1 << (g.logT - 1)) + 1) & ~1));
+  return sizeof(float2) * ((size_t)D * (1 << g.logP) + ((size_t)1 << g.logT));
 }
 
 template <typename K>
@@ -327,6 +679,20 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 bool nd_aligned16(const void* q) { return q && ((reinterpret_cast<uintptr_t>(q) & 15u) == 0); }
+
+template <typename T>
+cudaError_t launch_nd(const void* v, const void* const* x, const SpecPtrs& kh, void* y, const NdGeom& g, int B, int D,
+                      int N, unsigned blocks, cudaStream_t s) {
+  NdGates<T> xs{};
+  for (int n = 0; n < N; ++n) xs.p[n] = reinterpret_cast<const T*>(x[n]);
+  const bool staged = nd_staged(g, sizeof(T));
+  const size_t smem = nd_smem(g, sizeof(T), staged);
+  auto kern = staged ? nd_forward_kernel<T, true> : nd_forward_kernel<T, false>;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<blocks, nd_threads(g), smem, s>>>(reinterpret_cast<const T*>(v), xs, kh, reinterpret_cast<T*>(y), g, B, D, N);
+  return cudaGetLastError();
+}
 
 }  // namespace
 
@@ -352,9 +718,9 @@ hyena_status hyena_nd_filter_spectrum(const float* K, int D, int nd, const int* 
   float2* out = reinterpret_cast<float2*>(khat);
   nd_table_kernel<<<1, 256, 0, s>>>(out + (size_t)D * (1 << g.logP), g.logT);
   cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) e = set_smem(nd_spectrum_kernel, nd_smem(g));
+  if (e == cudaSuccess) e = set_smem(nd_spectrum_kernel, nd_spec_smem(g));
   if (e == cudaSuccess) {
-    nd_spectrum_kernel<<<D, nd_threads(g), nd_smem(g), s>>>(K, out, g, D);
+    nd_spectrum_kernel<<<D, nd_threads(g), nd_spec_smem(g), s>>>(K, out, g, D);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? HYENA_OK : report_cuda_error(e);
@@ -374,28 +740,10 @@ hyena_status hyena_nd_forward(const void* v, const void* const* x, const void* c
   if (blocks > 0x7fffffffLL) return HYENA_ERR_INVALID_ARG;
   SpecPtrs kh{};
   for (int n = 0; n < N; ++n) kh.p[n] = reinterpret_cast<const float2*>(khat[n]);
-  cudaStream_t s = (cudaStream_t)stream;
-  const size_t smem = nd_smem(g);
-  cudaError_t e;
-  if (dtype == HYENA_BF16) {
-    NdGates<__nv_bfloat16> xs{};
-    for (int n = 0; n < N; ++n) xs.p[n] = reinterpret_cast<const __nv_bfloat16*>(x[n]);
-    e = set_smem(nd_forward_kernel<__nv_bfloat16>, smem);
-    if (e == cudaSuccess) {
-      nd_forward_kernel<__nv_bfloat16><<<(unsigned)blocks, nd_threads(g), smem, s>>>(
-          reinterpret_cast<const __nv_bfloat16*>(v), xs, kh, reinterpret_cast<__nv_bfloat16*>(y), g, B, D, N);
-      e = cudaGetLastError();
-    }
-  } else {
-    NdGates<float> xs{};
-    for (int n = 0; n < N; ++n) xs.p[n] = reinterpret_cast<const float*>(x[n]);
-    e = set_smem(nd_forward_kernel<float>, smem);
-    if (e == cudaSuccess) {
-      nd_forward_kernel<float><<<(unsigned)blocks, nd_threads(g), smem, s>>>(
-          reinterpret_cast<const float*>(v), xs, kh, reinterpret_cast<float*>(y), g, B, D, N);
-      e = cudaGetLastError();
-    }
-  }
+  const cudaError_t e = dtype == HYENA_BF16 ? launch_nd<__nv_bfloat16>(v, x, kh, y, g, B, D, N, (unsigned)blocks,
+                                                                       (cudaStream_t)stream)
+                                            : launch_nd<float>(v, x, kh, y, g, B, D, N, (unsigned)blocks,
+                                                               (cudaStream_t)stream);
   return e == cudaSuccess ? HYENA_OK : report_cuda_error(e);
 }
 

@@ -167,10 +167,11 @@ def test_f16_spectra_queries_and_host_rejections(lib):
 def test_nd_queries_and_host_rejections(lib):
     p, mis = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
     I3 = ctypes.c_int * 3
-    # [D][P] float2 then the twiddle table (half the longest padded axis, even count)
-    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(64, 64, 0), 0) == 8 * (4 * 128 * 128 + 64)
-    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(128, 128, 0), 1) == 8 * (4 * 128 * 128 + 64)
+    # [D][P] float2 then the twiddle table (one entry per point of the longest padded axis, at least 2)
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(64, 64, 0), 0) == 8 * (4 * 128 * 128 + 128)
+    assert lib.hyena_nd_spectrum_bytes(4, 2, I3(128, 128, 0), 1) == 8 * (4 * 128 * 128 + 128)
     assert lib.hyena_nd_spectrum_bytes(1, 3, I3(2, 2, 2), 1) == 8 * (8 + 2)
+    assert lib.hyena_nd_spectrum_bytes(1, 1, I3(1, 0, 0), 1) == 8 * (1 + 2)
     assert lib.hyena_nd_spectrum_bytes(4, 2, I3(128, 128, 0), 0) == 0      # padded grid above 16384 points
     assert lib.hyena_nd_spectrum_bytes(4, 1, I3(1024, 0, 0), 0) == 0       # padded axis above 1024
     assert lib.hyena_nd_spectrum_bytes(4, 2, I3(12, 16, 0), 0) == 0        # not a power of two

@@ -59,6 +59,9 @@ SHAPES = [
     (2, "f32", 2, 2, (4, 8, 8), "zero"),
     (2, "f32", 2, 2, (8, 4, 16), "circular"),
     (1, "f32", 2, 1, (2, 2, 2), "circular"),
+    (2, "f32", 2, 2, (1, 64), "circular"),     # unit axes are dropped
+    (2, "f32", 1, 2, (8, 1, 16), "circular"),
+    (2, "f32", 3, 1, (1, 1, 1), "circular"),   # a single point: y = x_N ... K^ v
     (2, "f32", 2, 2, (64, 64), "zero"),
     (2, "f32", 1, 2, (128, 128), "circular"),
     (2, "f32", 2, 1, (512,), "zero"),          # longest padded axis (1024)
