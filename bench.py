@@ -15,6 +15,11 @@ and the fraction of the HBM roofline; one JSON line is printed by rank 0.
 (weak scaling, no collective on the data path); time is the max over ranks.
 --impl reference times the float64 CPU oracle on a bounded sample of the
 same workload (rank 0 only).
+The e2e figure times steps through the public API with every step's inputs
+copied in from pinned host memory and its result copied back; forward,
+striped and ND steps rotate over three CUDA streams so that one step's
+copies overlap its neighbours' kernels (the backward, which shares one
+workspace, runs its steps on one stream).
 --pass backward times hyena_backward instead (dv, dx_n and dh_n from a loss
 gradient dy), same workload and conventions; its roofline counts the bytes
 the gradients must move at least: v, x_n, dy and the spectra in, dv, dx_n
@@ -285,6 +290,53 @@ def oracle_striped_sample(w: synth.Workload, target_core_seconds: float = 8.0):
                       f"direct FIR sums", "seconds": dt}
 
 
+E2E_SLOTS = 3
+
+
+def pipelined_e2e(torch, dev, main_stream, pinned_in, make_slot, steps, world, dist):
+    """Device time (ms, max over ranks) of `steps` end-to-end steps through the
+    public API, rotated over E2E_SLOTS CUDA streams: step i runs on slot
+    i % E2E_SLOTS and copies its pinned host inputs into that slot's device
+    buffers, makes the library call, and copies the result into that slot's
+    pinned host buffers. Every step moves all of its inputs in and its result
+    out; the rotation lets one step's uploads overlap its neighbours' kernels
+    and downloads (each direction has its own copy engine).
+    make_slot(stream) -> (device input tensors, call returning the outputs,
+    pinned host output tensors)."""
+    slots = []
+    for _ in range(E2E_SLOTS):
+        st = torch.cuda.Stream(device=dev)
+        slots.append((st, make_slot(st)))
+
+    def step(i):
+        st, (dins, call, pouts) = slots[i % E2E_SLOTS]
+        with torch.cuda.stream(st):
+            for d, p in zip(dins, pinned_in):
+                d.copy_(p, non_blocking=True)
+            for p, o in zip(pouts, call()):
+                p.copy_(o, non_blocking=True)
+
+    for i in range(3 * E2E_SLOTS):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(main_stream)
+    for st, _ in slots:
+        st.wait_event(e0)
+    for i in range(steps):
+        step(i)
+    for st, _ in slots:
+        done = torch.cuda.Event()
+        done.record(st)
+        main_stream.wait_event(done)
+    e1.record(main_stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+
+
 def oracle_nd_sample(w: "synth.NDWorkload", target_core_seconds: float = 8.0):
     """The float64 HyenaND oracle (numpy FFT, one thread) on a bounded sample of rows."""
     import oracle
@@ -394,33 +446,15 @@ def run_nd(args) -> int:
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
 
     # end to end: pinned host inputs in, y out, through the same public call
-    pin_v = base_v.cpu().pin_memory()
-    pin_x = [x.cpu().pin_memory() for x in base_x]
-    dv = torch.empty_like(base_v)
-    dxs = [torch.empty_like(x) for x in base_x]
-    pin_y = torch.empty_like(pin_v).pin_memory()
-    e2e_call = hy.PreparedND(dv, dxs, base_k, w.dims, w.boundary, stream=stream)
+    pinned_in = [base_v.cpu().pin_memory()] + [x.cpu().pin_memory() for x in base_x]
 
-    def e2e_step():
-        dv.copy_(pin_v, non_blocking=True)
-        for d, p in zip(dxs, pin_x):
-            d.copy_(p, non_blocking=True)
-        pin_y.copy_(e2e_call(), non_blocking=True)
+    def nd_slot(st):
+        dv = torch.empty_like(base_v)
+        dxs = [torch.empty_like(x) for x in base_x]
+        call = hy.PreparedND(dv, dxs, base_k, w.dims, w.boundary, stream=st)
+        return [dv, *dxs], lambda: [call()], [torch.empty_like(pinned_in[0]).pin_memory()]
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    e2e_ms = pipelined_e2e(torch, dev, stream, pinned_in, nd_slot, args.e2e_steps, world, dist)
     e2e_value = whole_job_throughput(args.e2e_steps * w.channels * w.grid, world, e2e_ms)
     line = None
     if rank == 0:
@@ -437,7 +471,8 @@ def run_nd(args) -> int:
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT_ND,
                     "h2d_bytes_per_step": (w.N + 1) * w.channels * w.grid * w.elem_bytes,
-                    "d2h_bytes_per_step": w.channels * w.grid * w.elem_bytes, "ms_per_step": e2e_ms / args.e2e_steps},
+                    "d2h_bytes_per_step": w.channels * w.grid * w.elem_bytes, "ms_per_step": e2e_ms / args.e2e_steps,
+                    "streams": E2E_SLOTS},
             "gpu_launches": K_steps * launches_per_step,
             "clocks": clocks,
         }
@@ -636,43 +671,48 @@ def main():
         h2d = (w.N + 2) * w.channels * w.L * w.elem_bytes
         d2h = (w.N + 1) * w.channels * w.L * w.elem_bytes + 4 * w.N * w.D * w.L
     elif striped:
-        pin_y = torch.empty_like(pin_v).pin_memory()
-        e2e_call = hy.PreparedStriped(dxs[0], dxs[1], dv, *sf, stream=stream)
         h2d = 3 * w.channels * w.L * w.elem_bytes
         d2h = w.channels * w.L * w.elem_bytes
     else:
-        pin_y = torch.empty_like(pin_v).pin_memory()
-        e2e_call = hy.PreparedForward(dv, dxs, sets[0]._keep[2], stream=stream, f16_spectra=spec16)
         h2d = (w.N + 1) * w.channels * w.L * w.elem_bytes
         d2h = w.channels * w.L * w.elem_bytes
+
+    def slot(st):
+        sv = torch.empty_like(base_v)
+        sxs = [torch.empty_like(x) for x in base_x]
+        if striped:
+            call = hy.PreparedStriped(sxs[0], sxs[1], sv, *sf, stream=st)
+        else:
+            call = hy.PreparedForward(sv, sxs, sets[0]._keep[2], stream=st, f16_spectra=spec16)
+        return [sv, *sxs], lambda: [call()], [torch.empty_like(pin_v).pin_memory()]
 
     def e2e_step():
         dv.copy_(pin_v, non_blocking=True)
         for d, p in zip(dxs, pin_x):
             d.copy_(p, non_blocking=True)
-        if bwd:
-            ddy.copy_(pin_dy, non_blocking=True)
-            gdv, gdxs, gdh = e2e_call()
-            for p, t in zip(pin_out, [gdv, *gdxs, gdh]):
-                p.copy_(t, non_blocking=True)
-        else:
-            y = e2e_call()
-            pin_y.copy_(y, non_blocking=True)
+        ddy.copy_(pin_dy, non_blocking=True)
+        gdv, gdxs, gdh = e2e_call()
+        for p, t in zip(pin_out, [gdv, *gdxs, gdh]):
+            p.copy_(t, non_blocking=True)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    if bwd:
+        # one workspace and one set of outputs: the steps run back to back on one stream
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
+    else:
+        e2e_ms = pipelined_e2e(torch, dev, stream, [pin_v, *pin_x], slot, args.e2e_steps, world, dist)
     e2e_value = whole_job_throughput(args.e2e_steps * w.channels * w.L, world, e2e_ms)
 
     line = None
@@ -694,7 +734,8 @@ def main():
                                     ("striped_kernel (fused FIR)" if striped else dominant_kernel(w, spec16)[0])),
                          "kernel_ms": round(kernel_ms, 5)},
             "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.e2e_steps,
+                    "streams": 1 if bwd else E2E_SLOTS},
             "gpu_launches": K * launches_per_step,
             "clocks": clocks,
         }
