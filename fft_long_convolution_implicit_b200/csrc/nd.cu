@@ -52,16 +52,16 @@ struct NdGeom {
   // blocks of 2^st_logm[i] points with radix 2^st_logR[i]
   int nsteps;
   signed char st_a[kNdMaxSteps], st_logm[kNdMaxSteps], st_logR[kNdMaxSteps];
+  // zero padding: step i skips the butterflies whose offset along the later
+  // axes lies in their padding (bit st_p1/st_p2 of the offset set; -1 = none),
+  // and the first step of an axis reads only the lower half of that axis
+  signed char st_p1[kNdMaxSteps], st_p2[kNdMaxSteps], st_first[kNdMaxSteps];
 };
 
 __device__ __forceinline__ float ld1(const float* p) { return __ldg(p); }
 __device__ __forceinline__ float ld1(const __nv_bfloat16* p) { return __bfloat162float(__ldg(p)); }
 __device__ __forceinline__ void st1(float* p, float v) { *p = v; }
 __device__ __forceinline__ void st1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
-
-// (-i) * a and (+i) * a
-__device__ __forceinline__ float2 mul_mi(float2 a) { return make_float2(a.y, -a.x); }
-__device__ __forceinline__ float2 mul_pi(float2 a) { return make_float2(-a.y, a.x); }
 
 // Padded-grid position of grid point g (row-major over L_0 x L_1 x L_2).
 __device__ __forceinline__ int grid_to_pos(const NdGeom& g, int gi) {
@@ -91,98 +91,6 @@ __device__ __forceinline__ int pos_to_grid(const NdGeom& g, int pos) {
   return gi;
 }
 
-// Spectrum kernel transform: 2-point levels, two at a time (same output order
-// as the radix steps of the forward kernel).
-// One radix-2 level (block size 2^logm) along an axis of inner stride 2^logs.
-template <bool INV>
-__device__ __forceinline__ void level2(float2* s, const float2* tw, int logT, int logm, int logs, int P, int tid,
-                                       int nt) {
-  const int logh = logm - 1;
-  for (int t = tid; t < (P >> 1); t += nt) {
-    const int in = t & ((1 << logs) - 1);
-    const int r = t >> logs;
-    const int j = r & ((1 << logh) - 1);
-    const int blk = r >> logh;
-    const int i0 = (((blk << logm) + j) << logs) + in;
-    const int i1 = i0 + (1 << (logh + logs));
-    const float2 w = tw[j << (logT - logm)];
-    const float2 a = s[i0], b = s[i1];
-    if (!INV) {
-      s[i0] = cadd(a, b);
-      s[i1] = cmul(csub(a, b), w);
-    } else {
-      const float2 bw = cmulc(b, w);
-      s[i0] = cadd(a, bw);
-      s[i1] = csub(a, bw);
-    }
-  }
-}
-
-// Two radix-2 levels (block sizes 2^logm and 2^(logm-1)) fused in registers.
-template <bool INV>
-__device__ __forceinline__ void level4(float2* s, const float2* tw, int logT, int logm, int logs, int P, int tid,
-                                       int nt) {
-  const int logq = logm - 2;
-  for (int t = tid; t < (P >> 2); t += nt) {
-    const int in = t & ((1 << logs) - 1);
-    const int r = t >> logs;
-    const int j = r & ((1 << logq) - 1);
-    const int blk = r >> logq;
-    const int i0 = (((blk << logm) + j) << logs) + in;
-    const int dq = 1 << (logq + logs);
-    const float2 w1 = tw[j << (logT - logm)];        // w_m^j
-    const float2 w2 = tw[j << (logT - logm + 1)];    // w_{m/2}^j
-    float2 x0 = s[i0], x1 = s[i0 + dq], x2 = s[i0 + 2 * dq], x3 = s[i0 + 3 * dq];
-    if (!INV) {
-      const float2 a0 = cadd(x0, x2), a2 = cmul(csub(x0, x2), w1);
-      const float2 a1 = cadd(x1, x3), a3 = cmul(mul_mi(csub(x1, x3)), w1);
-      s[i0] = cadd(a0, a1);
-      s[i0 + dq] = cmul(csub(a0, a1), w2);
-      s[i0 + 2 * dq] = cadd(a2, a3);
-      s[i0 + 3 * dq] = cmul(csub(a2, a3), w2);
-    } else {
-      const float2 t1 = cmulc(x1, w2), t3 = cmulc(x3, w2);
-      const float2 a0 = cadd(x0, t1), a1 = csub(x0, t1);
-      const float2 a2 = cadd(x2, t3), a3 = csub(x2, t3);
-      const float2 u2 = cmulc(a2, w1), u3 = mul_pi(cmulc(a3, w1));
-      s[i0] = cadd(a0, u2);
-      s[i0 + 2 * dq] = csub(a0, u2);
-      s[i0 + dq] = cadd(a1, u3);
-      s[i0 + 3 * dq] = csub(a1, u3);
-    }
-  }
-}
-
-// Forward transform (natural order in, per-axis bit-reversed out) or its
-// inverse (bit-reversed in, natural out, scaled by P). Ends with a barrier.
-template <bool INV>
-__device__ void nd_transform(float2* s, const float2* tw, const NdGeom& g, int tid, int nt) {
-  const int P = 1 << g.logP;
-  for (int a = 0; a < g.nd; ++a) {
-    const int n = g.logn[a], ls = g.logs[a];
-    const bool odd = n & 1;
-    if (!INV) {
-      if (odd) {
-        level2<false>(s, tw, g.logT, n, ls, P, tid, nt);
-        __syncthreads();
-      }
-      for (int m = odd ? n - 1 : n; m >= 2; m -= 2) {
-        level4<false>(s, tw, g.logT, m, ls, P, tid, nt);
-        __syncthreads();
-      }
-    } else {
-      for (int m = 2; m <= (odd ? n - 1 : n); m += 2) {
-        level4<true>(s, tw, g.logT, m, ls, P, tid, nt);
-        __syncthreads();
-      }
-      if (odd) {
-        level2<true>(s, tw, g.logT, n, ls, P, tid, nt);
-        __syncthreads();
-      }
-    }
-  }
-}
-
 template <typename T>
 struct NdGates {
   const T* p[kMaxOrder];
@@ -208,13 +116,30 @@ constexpr int log2_of() {
 // axis of inner stride 2^logs (read once per pass from the shared geometry).
 struct StepGeo {
   int logs, logq, logm;
+  int nskip, p1, p2;   // skipped offset bits (ascending), their count
+  bool half_in;        // forward: inputs of the upper half of the axis are zero
 };
+// ZP: zero-padded boundary (pruning on); circular grids compile without it.
+template <bool ZP>
 __device__ __forceinline__ StepGeo step_geo(const NdGeom& g, int i) {
   StepGeo q;
   q.logm = g.st_logm[i];
   q.logq = q.logm - g.st_logR[i];
   q.logs = g.logs[g.st_a[i]];
+  q.p1 = ZP ? g.st_p1[i] : -1;
+  q.p2 = ZP ? g.st_p2[i] : -1;
+  q.nskip = ZP ? (q.p1 >= 0) + (q.p2 >= 0) : 0;
+  q.half_in = ZP && g.zero && g.st_first[i];
   return q;
+}
+
+// Butterfly index of the tc-th butterfly that is not skipped: zero bits
+// inserted at the skipped positions (lower one first).
+__device__ __forceinline__ int ins0(int x, int p) { return ((x >> p) << (p + 1)) | (x & ((1 << p) - 1)); }
+__device__ __forceinline__ int expand_t(const StepGeo& q, int tc) {
+  if (q.p1 >= 0) tc = ins0(tc, q.p1);
+  if (q.p2 >= 0) tc = ins0(tc, q.p2);
+  return tc;
 }
 
 // Butterfly t: positions base + r * stride (r < R) in the padded grid;
@@ -287,17 +212,18 @@ __device__ __forceinline__ void dit(float2 (&a)[R], const float2* tw, int logT, 
   dftR<R, true, 0>(a);
 }
 
-template <int R, bool INV>
+template <int R, bool INV, bool ZP>
 __device__ void plain_step(float2* s, const float2* tw, const NdGeom& g, int i, int tid, int nt) {
   constexpr int LR = log2_of<R>();
-  const StepGeo q = step_geo(g, i);
-  const int nb = (1 << g.logP) >> LR, logT = g.logT;
-  for (int t = tid; t < nb; t += nt) {
-    const StepIdx x = step_index(q, t);
+  const StepGeo q = step_geo<ZP>(g, i);
+  const int nb = ((1 << g.logP) >> LR) >> q.nskip, logT = g.logT;
+  for (int tc = tid; tc < nb; tc += nt) {
+    const StepIdx x = step_index(q, expand_t(q, tc));
     float2 a[R];
     if (!INV) {
 #pragma unroll
-      for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + r * x.stride)];
+      for (int r = 0; r < R; ++r)
+        a[r] = (q.half_in && r >= R / 2) ? make_float2(0.f, 0.f) : s[spad(x.base + r * x.stride)];
       dif<R>(a, tw, logT, x);
 #pragma unroll
       for (int r = 0; r < R; ++r) s[spad(x.base + brev_bits(r, LR) * x.stride)] = a[r];
@@ -316,11 +242,11 @@ __device__ void plain_step(float2* s, const float2* tw, const NdGeom& g, int i, 
 // runs along the innermost axis with one butterfly per block, so its R points
 // are contiguous (stride 1): their spectrum values are fetched first, as
 // 16-byte loads, to overlap the forward DFT.
-template <int R>
+template <int R, bool ZP>
 __device__ void turn_step(float2* s, const float2* tw, const NdGeom& g, int i, const float2* __restrict__ H, int tid,
                           int nt) {
   constexpr int LR = log2_of<R>();
-  const StepGeo q = step_geo(g, i);
+  const StepGeo q = step_geo<ZP>(g, i);   // innermost axis: nothing to skip
   const int nb = (1 << g.logP) >> LR, logT = g.logT;
   for (int t = tid; t < nb; t += nt) {
     const StepIdx x = step_index(q, t);
@@ -334,7 +260,7 @@ __device__ void turn_step(float2* s, const float2* tw, const NdGeom& g, int i, c
     }
     float2 a[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) a[r] = s[spad(x.base + r)];
+    for (int r = 0; r < R; ++r) a[r] = (q.half_in && r >= R / 2) ? make_float2(0.f, 0.f) : s[spad(x.base + r)];
     dif<R>(a, tw, logT, x);
 #pragma unroll
     for (int r = 0; r < R; ++r) a[r] = cmul(a[r], hk[brev_bits(r, LR)]);
@@ -365,21 +291,15 @@ struct PairSrc {
 // Steps 0 run along axis 0 over whole axes (one block), so butterfly t holds
 // axis-0 coordinates j + r q at the inner offset in: the grid index is
 // (j + r q) * (G / L_0) + inner_to_grid(in) inside the grid.
-struct Axis0Map {
-  int gin;        // grid index of the inner offset, -1 in the padding
-  int gstride;    // G / L_0
-  int L0;
-};
-
 // First forward step of stage 1 straight from v.
-template <int R, typename T, bool STAGED>
+template <int R, typename T, bool STAGED, bool ZP>
 __device__ void entry_step(float2* s, const float2* tw, const NdGeom& g, PairSrc<T, STAGED> src, int tid, int nt) {
   constexpr int LR = log2_of<R>();
-  const StepGeo q = step_geo(g, 0);
-  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  const StepGeo q = step_geo<ZP>(g, 0);
+  const int nb = ((1 << g.logP) >> LR) >> q.nskip, logT = g.logT;
   const int L0 = 1 << g.logL[0], gstride = g.G >> g.logL[0], qn = 1 << q.logq;
-  for (int t = tid; t < nb; t += nt) {
-    const StepIdx x = step_index(q, t);
+  for (int tc = tid; tc < nb; tc += nt) {
+    const StepIdx x = step_index(q, expand_t(q, tc));
     const int gin = inner_to_grid(g, x.in);
     float2 a[R];
 #pragma unroll
@@ -395,15 +315,15 @@ __device__ void entry_step(float2* s, const float2* tw, const NdGeom& g, PairSrc
 
 // Last inverse step of a stage, the gate x_n, then either the next stage's
 // first forward step (same positions) or the store of y.
-template <int R, bool LAST, typename T, bool STAGED>
+template <int R, bool LAST, typename T, bool STAGED, bool ZP>
 __device__ void exit_step(float2* s, const float2* tw, const NdGeom& g, PairSrc<T, STAGED> xg, T* __restrict__ y,
                           size_t row0, size_t row1, int tid, int nt) {
   constexpr int LR = log2_of<R>();
-  const StepGeo q = step_geo(g, 0);
-  const int nb = (1 << g.logP) >> LR, logT = g.logT;
+  const StepGeo q = step_geo<ZP>(g, 0);
+  const int nb = ((1 << g.logP) >> LR) >> q.nskip, logT = g.logT;
   const int L0 = 1 << g.logL[0], gstride = g.G >> g.logL[0], qn = 1 << q.logq;
-  for (int t = tid; t < nb; t += nt) {
-    const StepIdx x = step_index(q, t);
+  for (int tc = tid; tc < nb; tc += nt) {
+    const StepIdx x = step_index(q, expand_t(q, tc));
     const int gin = inner_to_grid(g, x.in);
     float2 a[R];
 #pragma unroll
@@ -451,7 +371,7 @@ __device__ __forceinline__ void stage_rows(T* dst, const T* __restrict__ src, si
   cp_async_commit();
 }
 
-template <typename T, bool STAGED>
+template <typename T, bool STAGED, bool ZP>
 __global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v, NdGates<T> xs, SpecPtrs kh,
                                                          T* __restrict__ y, NdGeom gp, int B, int D, int N) {
   // the step tables are indexed at run time: read them from shared memory
@@ -488,7 +408,7 @@ __global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v
   };
 
   if (F >= 2) {
-    ND_RADIX_SWITCH(g.st_logR[0], (entry_step<R, T, STAGED>(s, tw, g, src_of(v), tid, nt)));
+    ND_RADIX_SWITCH(g.st_logR[0], (entry_step<R, T, STAGED, ZP>(s, tw, g, src_of(v), tid, nt)));
   } else {
     const PairSrc<T, STAGED> vs = src_of(v);
     for (int i = tid; i < P; i += nt) {
@@ -505,17 +425,17 @@ __global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v
     // the gate rows arrive while the transform runs
     if (STAGED) stage_rows(xb, x_n, row0, row1, has1, G, tid, nt);
     for (int i = 1; i + 1 < F; ++i) {
-      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, false>(s, tw, g, i, tid, nt)));
+      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, false, ZP>(s, tw, g, i, tid, nt)));
       __syncthreads();
     }
     if (F >= 1) {
-      ND_RADIX_SWITCH(g.st_logR[F - 1], (turn_step<R>(s, tw, g, F - 1, H, tid, nt)));
+      ND_RADIX_SWITCH(g.st_logR[F - 1], (turn_step<R, ZP>(s, tw, g, F - 1, H, tid, nt)));
     } else {
       for (int i = tid; i < P; i += nt) s[spad(i)] = cmul(s[spad(i)], __ldg(H + i));
     }
     __syncthreads();
     for (int i = F - 2; i >= 1; --i) {
-      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, true>(s, tw, g, i, tid, nt)));
+      ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, true, ZP>(s, tw, g, i, tid, nt)));
       __syncthreads();
     }
     if (STAGED) {
@@ -525,9 +445,9 @@ __global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v
     const PairSrc<T, STAGED> xg = src_of(x_n);
     if (F >= 2) {
       if (last) {
-        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, true, T, STAGED>(s, tw, g, xg, y, row0, row1, tid, nt)));
+        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, true, T, STAGED, ZP>(s, tw, g, xg, y, row0, row1, tid, nt)));
       } else {
-        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, false, T, STAGED>(s, tw, g, xg, y, row0, row1, tid, nt)));
+        ND_RADIX_SWITCH(g.st_logR[0], (exit_step<R, false, T, STAGED, ZP>(s, tw, g, xg, y, row0, row1, tid, nt)));
       }
     } else {
       for (int i = tid; i < P; i += nt) {
@@ -550,25 +470,32 @@ __global__ void __launch_bounds__(512) nd_forward_kernel(const T* __restrict__ v
 }
 
 // Spectrum of one filter: K [D][grid] float32 -> [D][P] float2 (transform
-// order, times 1/P), one CTA per channel; the twiddle table follows.
-__global__ void __launch_bounds__(1024) nd_spectrum_kernel(const float* __restrict__ K, float2* __restrict__ out,
-                                                           NdGeom g, int D) {
+// order, times 1/P), one CTA per channel, with the forward kernel's radix
+// steps and shared-memory layout; the twiddle table follows the spectra.
+__global__ void __launch_bounds__(512) nd_spectrum_kernel(const float* __restrict__ K, float2* __restrict__ out,
+                                                          NdGeom gp, int D) {
+  __shared__ NdGeom g;
+  if (threadIdx.x == 0) g = gp;
   extern __shared__ float4 nd_smem_raw[];
   float2* s = reinterpret_cast<float2*>(nd_smem_raw);
-  const int P = 1 << g.logP;
-  float2* tw = s + P;
+  const int P = 1 << gp.logP;
+  float2* tw = s + spad(P) + 1;
   const int tid = threadIdx.x, nt = blockDim.x;
   const int c = blockIdx.x;
   const float2* tsrc = out + (size_t)D * P;
-  for (int i = tid; i < (1 << (g.logT - 1)); i += nt) tw[i] = tsrc[i];
-  for (int i = tid; i < P; i += nt) s[i] = make_float2(0.f, 0.f);
+  for (int i = tid; i < (1 << gp.logT); i += nt) tw[i] = tsrc[i];
+  for (int i = tid; i < P; i += nt) {
+    const int gi = pos_to_grid(gp, i);
+    s[spad(i)] = make_float2(gi < 0 ? 0.f : __ldg(K + (size_t)c * gp.G + gi), 0.f);
+  }
   __syncthreads();
-  for (int gi = tid; gi < g.G; gi += nt) s[grid_to_pos(g, gi)] = make_float2(__ldg(K + (size_t)c * g.G + gi), 0.f);
-  __syncthreads();
-  nd_transform<false>(s, tw, g, tid, nt);
+  for (int i = 0; i < gp.nsteps; ++i) {
+    ND_RADIX_SWITCH(g.st_logR[i], (plain_step<R, false, true>(s, tw, g, i, tid, nt)));
+    __syncthreads();
+  }
   const float inv = 1.0f / (float)P;   // exact: P is a power of two
   for (int i = tid; i < P; i += nt) {
-    const float2 u = s[i];
+    const float2 u = s[spad(i)];
     out[(size_t)c * P + i] = make_float2(u.x * inv, u.y * inv);
   }
 }
@@ -632,6 +559,12 @@ bool nd_geometry(int nd, const int* dims, int boundary, NdGeom* g) {
       r.st_a[r.nsteps] = (signed char)a;
       r.st_logm[r.nsteps] = (signed char)logm;
       r.st_logR[r.nsteps] = (signed char)lr;
+      r.st_first[r.nsteps] = (signed char)(q == 0);
+      int p[2] = {-1, -1}, np = 0;
+      if (r.zero)
+        for (int b = nd - 1; b > a; --b) p[np++] = r.logs[b] + r.logL[b];   // ascending
+      r.st_p1[r.nsteps] = (signed char)p[0];
+      r.st_p2[r.nsteps] = (signed char)p[1];
       ++r.nsteps;
       logm -= lr;
     }
@@ -664,10 +597,8 @@ size_t nd_smem(const NdGeom& g, size_t elem, bool staged) {
 bool nd_staged(const NdGeom& g, size_t elem) {
   return (elem * (size_t)g.G) % 16 == 0 && nd_smem(g, elem, true) + sizeof(NdGeom) <= (size_t)227 * 1024;
 }
-// spectrum kernel: unpadded grid, then half the table
-size_t nd_spec_smem(const NdGeom& g) {
-  return sizeof(float2) * (((size_t)1 << g.logP) + ((size_t)1 << (g.logT - 1)));
-}
+// spectrum kernel: the forward kernel's grid and table
+size_t nd_spec_smem(const NdGeom& g) { return nd_smem(g, 0, false); }
 
 size_t nd_block_bytes(const NdGeom& g, int D) {
   return sizeof(float2) * ((size_t)D * (1 << g.logP) + ((size_t)1 << g.logT));
@@ -687,7 +618,8 @@ cudaError_t launch_nd(const void* v, const void* const* x, const SpecPtrs& kh, v
   for (int n = 0; n < N; ++n) xs.p[n] = reinterpret_cast<const T*>(x[n]);
   const bool staged = nd_staged(g, sizeof(T));
   const size_t smem = nd_smem(g, sizeof(T), staged);
-  auto kern = staged ? nd_forward_kernel<T, true> : nd_forward_kernel<T, false>;
+  auto kern = g.zero ? (staged ? nd_forward_kernel<T, true, true> : nd_forward_kernel<T, false, true>)
+                     : (staged ? nd_forward_kernel<T, true, false> : nd_forward_kernel<T, false, false>);
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   kern<<<blocks, nd_threads(g), smem, s>>>(reinterpret_cast<const T*>(v), xs, kh, reinterpret_cast<T*>(y), g, B, D, N);
