@@ -261,7 +261,51 @@ __device__ __forceinline__ void fir8T(const float* f, int len, const T* x, int p
   }
 }
 
+// Eight consecutive staged elements as floats, from one 16-byte (bf16) or two
+// (float) aligned shared-memory loads.
 template <typename T>
+__device__ __forceinline__ void load8f(const T* p, float* w);
+template <>
+__device__ __forceinline__ void load8f<__nv_bfloat16>(const __nv_bfloat16* p, float* w) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    w[2 * k] = __uint_as_float(v[k] << 16);
+    w[2 * k + 1] = __uint_as_float(v[k] & 0xffff0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load8f<float>(const float* p, float* w) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+}
+
+// acc[p] = sum_{j < LEN} f[j] x[pos + p - j] for a compile-time LEN <= 9:
+// the 16 points pos-8 .. pos+7 come from two aligned vector loads and every
+// tap is unrolled (pos a multiple of 8 elements, 16-byte aligned).
+template <typename T, int LEN>
+__device__ __forceinline__ void fir8v(const float* f, const T* x, int pos, float (&acc)[kStPer]) {
+  static_assert(LEN >= 1 && LEN <= 9, "fir8v covers up to 9 taps");
+  float w[16];
+  load8f<T>(x + pos - 8, w);
+  load8f<T>(x + pos, w + 8);
+  float g[LEN];
+#pragma unroll
+  for (int j = 0; j < LEN; ++j) g[j] = f[j];
+#pragma unroll
+  for (int p = 0; p < kStPer; ++p) {
+    float a = 0.f;
+#pragma unroll
+    for (int j = 0; j < LEN; ++j) a = fmaf(g[j], w[8 + p - j], a);
+    acc[p] = a;
+  }
+}
+
+// LFC, LGC > 0: filter lengths fixed at compile time (the Hyena-SE sizes),
+// taps unrolled over vector-loaded windows; 0: any length (sliding windows).
+template <typename T, int LFC, int LGC>
 __global__ void __launch_bounds__(kStThreads)
 striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __restrict__ xv,
                     const float* __restrict__ hT, const float* __restrict__ hH, const float* __restrict__ hK, int lf,
@@ -273,7 +317,8 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
   const int hg = lg - 1, hf = lf - 1, Hx = hg + hf;
   const int HP = ((Hx + V - 1) / V) * V;           // halo slots, 16-byte multiple
   const int W = HP + kStTile;                       // elements per staged window
-  const int Pu = pad4(hg);
+  // u row offset; the vector windows of fir8v read 8 slots before each output
+  const int Pu = LGC > 0 ? max(pad4(hg), 8) : pad4(hg);
   const int S = pad4(kStTile + lg + 24);
   const size_t winb = ((size_t)W * E + 127) & ~(size_t)127;
   // [stage][xq, xk, xv] windows, then su (float), filters, mbarriers
@@ -348,10 +393,18 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
     const int base = tid * kStPer;
     if (base < n_out) {
       float a[kStPer], b[kStPer];
-      fir8T<T>(fH, lf, wk, HP + base, a);
-      fir8T<T>(fK, lf, wv, HP + base, b);
+      if constexpr (LFC > 0) {
+        fir8v<T, LFC>(fH, wk, HP + base, a);
+        fir8v<T, LFC>(fK, wv, HP + base, b);
+        float4* su4 = reinterpret_cast<float4*>(su + Pu + base);
+        su4[0] = make_float4(a[0] * b[0], a[1] * b[1], a[2] * b[2], a[3] * b[3]);
+        su4[1] = make_float4(a[4] * b[4], a[5] * b[5], a[6] * b[6], a[7] * b[7]);
+      } else {
+        fir8T<T>(fH, lf, wk, HP + base, a);
+        fir8T<T>(fK, lf, wv, HP + base, b);
 #pragma unroll
-      for (int p = 0; p < kStPer; ++p) su[Pu + base + p] = a[p] * b[p];
+        for (int p = 0; p < kStPer; ++p) su[Pu + base + p] = a[p] * b[p];
+      }
     }
     for (int i = tid; i < hg; i += kStThreads) {
       const int t = t0 - hg + i;
@@ -365,8 +418,13 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
     __syncthreads();
     if (base < n_out) {
       float q[kStPer], out[kStPer];
-      fir8T<T>(fT, lf, wq, HP + base, q);
-      fir8(fG, lg, su, Pu + base, out);
+      if constexpr (LFC > 0) {
+        fir8v<T, LFC>(fT, wq, HP + base, q);
+        fir8v<float, LGC>(fG, su, Pu + base, out);
+      } else {
+        fir8T<T>(fT, lf, wq, HP + base, q);
+        fir8(fG, lg, su, Pu + base, out);
+      }
 #pragma unroll
       for (int p = 0; p < kStPer; ++p) out[p] *= q[p];
       T* dst = y + (size_t)rowi * L + t0 + base;
@@ -408,7 +466,7 @@ size_t striped_bulk_smem(int E, int lf, int lg) {
   const int V = 16 / E, Hx = lg - 1 + lf - 1;
   const size_t HP = (size_t)((Hx + V - 1) / V) * V;
   const size_t winb = ((HP + kStTile) * E + 127) & ~(size_t)127;
-  const size_t S = (size_t)((kStTile + lg + 24 + 3) & ~3);
+  const size_t S = (size_t)((kStTile + lg + 24 + 3) & ~3);   // u row: offset (<= max(pad4(lg-1), 8)) + tile
   return 6 * winb + sizeof(float) * (S + 48 + (size_t)((lg + 3) & ~3) + 4) + 2 * sizeof(uint64_t);
 }
 
@@ -416,7 +474,8 @@ template <typename T>
 cudaError_t launch_striped_bulk(const void* xq, const void* xk, const void* xv, const float* hT, const float* hH,
                                 const float* hK, int lf, const float* hG, int lg, int B, int D, int L, void* y,
                                 cudaStream_t s) {
-  auto k = striped_bulk_kernel<T>;
+  // the Hyena-SE sizes (featurizers of 4 taps, inner filter of 7) take the unrolled kernel
+  auto k = (lf == 4 && lg == 7) ? striped_bulk_kernel<T, 4, 7> : striped_bulk_kernel<T, 0, 0>;
   const size_t smem = striped_bulk_smem((int)sizeof(T), lf, lg);
   int grid = 0;
   cudaError_t e = persistent_grid((const void*)k, kStThreads, smem, &grid);

@@ -47,6 +47,8 @@ SHAPES = [
     ("bf16", 2, 3, 100, 4, 7),
     ("f32", 1, 2, 5000, 7, 5),       # three tiles, ragged tail
     ("bf16", 4, 8, 2048, 4, 7),
+    ("f32", 1, 2, 5000, 4, 7),       # SE sizes on the unrolled kernel: three tiles, ragged tail
+    ("bf16", 2, 2, 6144, 4, 7),
     ("f32", 2, 2, 4096, 3, 128),     # MR
     ("bf16", 1, 3, 6000, 5, 1024),   # longest inner filter, halo past a tile
     ("f32", 1, 1, 1, 1, 1),          # degenerate
