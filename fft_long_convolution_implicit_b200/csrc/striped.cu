@@ -22,6 +22,10 @@ namespace {
 constexpr int kStThreads = 256;
 constexpr int kStTile = 2048;        // outputs per CTA
 constexpr int kStPer = kStTile / kStThreads;   // consecutive outputs per thread (8)
+// The bulk kernel zero-fills the halo of a row's first tile only (t0 < halo);
+// every later tile must start at least one full halo into the row.
+static_assert(kStTile >= ((kMaxStripedLG - 1 + kMaxStripedLF - 1 + 7) / 8) * 8,
+              "a tile must be at least as long as the longest staged halo");
 
 template <typename T>
 __device__ __forceinline__ float ld1(const T* p);
