@@ -3,7 +3,8 @@
 //
 // The causal long convolution of the Hyena operator is evaluated by FFT on
 // a 2L zero-padded grid (glossary "Hyena（ハイエナ）", section 計算効率;
-// HyenaND summary, 境界の処理). A length-2L real sequence z is packed as
+// "Native Multi-Dimensional Subquadratic Operators via Input Dependent Long
+// Convolutions", section 境界の処理). A length-2L real sequence z is packed as
 // M = L complex points c[m] = z[2m] + i z[2m+1]; its upper half is zero.
 // The M-point complex FFT is an in-place Stockham autosort FFT in shared
 // memory: forward pass p with radix R and span Ns reads butterfly j at

@@ -1,8 +1,9 @@
 // nd.cu -- HyenaND: the order-N recurrence with an N-dimensional global
-// convolution (HyenaND summary, section 手法: the convolution runs on the
-// L_1 x ... x L_N grid through an N-dimensional FFT, circular for periodic
-// data, or on the input zero-padded to twice the grid so nothing leaks across
-// the boundary).
+// convolution (page "Native Multi-Dimensional Subquadratic Operators via
+// Input Dependent Long Convolutions", section 手法: the convolution runs on
+// the L_1 x ... x L_N grid through an N-dimensional FFT, circular for
+// periodic data, or on the input zero-padded to twice the grid so nothing
+// leaks across the boundary).
 //
 //   z_1 = v,  z_{n+1} = x_n (.) (K_n conv z_n),  y = z_{N+1}
 //   circular: (K conv z)[p] = sum_q K[(p - q) mod dims] z[q]

@@ -7,7 +7,8 @@
 // As in the mma.sync kernel, batch items b, b+1 of channel c share h_c, so
 // their causal convolutions are the real and imaginary parts of one complex
 // convolution of c[n] = z_b[n] + i z_{b+1}[n] on the 2L zero-padded grid
-// (glossary "Hyena（ハイエナ）", section 計算効率; HyenaND summary, 境界の処理).
+// (glossary "Hyena（ハイエナ）", section 計算効率; "Native Multi-Dimensional
+// Subquadratic Operators via Input Dependent Long Convolutions", section 境界の処理).
 // The 4096-point transform runs as three radix-16 DFT passes, each one GEMM
 // D[256 x 32] = A[256 x K] B[32 x K]^T on the tensor cores:
 //   n = 256 a + 16 b + c,  k = d + 16 e + 256 f

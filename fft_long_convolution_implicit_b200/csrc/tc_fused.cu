@@ -4,7 +4,8 @@
 // Two batch items b, b+1 of one channel c share the filter h_c, so their
 // causal convolutions are the real and imaginary parts of one complex
 // convolution: c[t] = z_b[t] + i z_{b+1}[t] on the 2L zero-padded grid
-// (glossary "Hyena（ハイエナ）", section 計算効率; HyenaND summary, 境界の処理).
+// (glossary "Hyena（ハイエナ）", section 計算効率; "Native Multi-Dimensional
+// Subquadratic Operators via Input Dependent Long Convolutions", section 境界の処理).
 // Its 2L-point transform is split 2L = R0 * 256, m = 256 n0 + m', bin
 // k = k0 + R0 k':
 //   outer  (fp32 SIMT, thread m'): DFT_R0 over n0, twiddle w_{2L}^{m' k0};

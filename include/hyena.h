@@ -11,7 +11,8 @@
  * where (.) is the elementwise product and * the causal long convolution
  * (h * z)_t = sum_{s=0..t} h_{t-s} z_s ("02. 3つの Hyena 演算子", section 4,
  * the FIR sum), evaluated by FFT on a 2L zero-padded grid (glossary
- * "Hyena（ハイエナ）", section 計算効率; HyenaND summary, 境界の処理).
+ * "Hyena（ハイエナ）", section 計算効率; "Native Multi-Dimensional Subquadratic
+ * Operators via Input Dependent Long Convolutions", section 境界の処理).
  * The filters are implicit (glossary "Hyena（ハイエナ）", section
  * 暗黙的畳み込みフィルタ: h(t) = Window(t) FFN(t/L, sin, cos)).
  *
@@ -169,9 +170,9 @@ hyena_status hyena_forward_static_workspace(const void *v, const void *const *x,
 
 /*
  * Reduced-precision filter spectra (no counterpart on the pages, which fix
- * no precision for the cached spectrum: page "Hyena Hierarchy ... long
- * convolution language models", section 計算方法, only states that the long
- * convolution runs through the FFT). The forward reads the spectrum of every
+ * no precision for the cached spectrum: page "Hyena Hierarchy: Towards
+ * Larger Convolutional Language Models", section 計算方法, only states that
+ * the long convolution runs through the FFT). The forward reads the spectrum of every
  * filter once per channel, and at D*L of that size the float32 spectrum is
  * the largest stream of a step; the f16 block halves it.
  *
@@ -327,7 +328,8 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
 hyena_status hyena_device_timeouts(void);
 
 /*
- * HyenaND (HyenaND summary, section 手法: a global convolution evaluated on
+ * HyenaND (page "Native Multi-Dimensional Subquadratic Operators via Input
+ * Dependent Long Convolutions", section 手法: a global convolution evaluated on
  * the L_1 x ... x L_nd grid through an nd-dimensional FFT; circular for
  * periodic data, or with the input zero-padded to twice the grid so that
  * nothing leaks across the boundary). The order-N recurrence of

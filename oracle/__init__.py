@@ -265,8 +265,9 @@ def exponential_filter(R, lam, L: int) -> np.ndarray:
 
 
 # ------------------------------------------------------------------ HyenaND --
-# The N-dimensional operator of the HyenaND summary (page "HyenaND ... nSubQ",
-# section 手法: a global convolution evaluated on the L_1 x ... x L_N grid
+# The N-dimensional operator of HyenaND (page "Native Multi-Dimensional
+# Subquadratic Operators via Input Dependent Long Convolutions", section 手法:
+# a global convolution evaluated on the L_1 x ... x L_N grid
 # itself through an N-dimensional FFT, with a circular boundary for periodic
 # systems or zero padding of the input to twice the grid for non-periodic
 # data). Plain numpy, float64; numpy's FFT is the only library step.

@@ -1,5 +1,6 @@
 """HyenaND parity: the CUDA path (through the C ABI) against the float64
-oracle's ND convolution recurrence (HyenaND summary, section 手法).
+oracle's ND convolution recurrence (page "Native Multi-Dimensional
+Subquadratic Operators via Input Dependent Long Convolutions", section 手法).
 
 Tolerance: per (b, c) row relative L2 <= 2e-5 for float32 I/O and <= 8e-3 for
 bfloat16 I/O, the bar of the 1-D forward (the same float32 transform

@@ -1,5 +1,6 @@
 """Pins of the HyenaND oracle (ND convolution, circular or zero-padded
-boundary; HyenaND summary, section 手法) to results fixed independently of
+boundary; page "Native Multi-Dimensional Subquadratic Operators via Input
+Dependent Long Convolutions", section 手法) to results fixed independently of
 its FFT evaluation: brute-force sums on tiny grids, delta and shifted-delta
 kernels, separable kernels against the 1D causal sum of the C oracle, the
 1D case against the 1D order-N oracle, and the no-wrap equivalence of the
