@@ -11,6 +11,12 @@ an exception is raised.
     y    = forward(v, [x1, ..., xN], hhat)                            # [B][D][L]
     dv, dxs, dh = backward(v, [x1, ..., xN], hhat, dy)                # gradients
     grads = filter_backward(weights, N, D, L, alpha_lo, alpha_hi, dh) # FFN weight gradients
+
+    h16  = [spectrum_to_f16(t, D, L) for t in hhat]                   # f16 spectra
+    y    = forward_f16_spectra(v, [x1, ..., xN], h16)
+    y    = striped_forward(xq, xk, xv, hT, hH, hK, hG)                # q . (hG * (k . v))
+    kh   = [nd_filter_spectrum(K[n], dims, "zero") for n in range(N)] # HyenaND kernels
+    y    = nd_forward(v, [x1, ..., xN], kh, dims, "zero")             # [B][D][*dims]
 """
 from __future__ import annotations
 

@@ -80,3 +80,25 @@ def test_sample_rows():
     s = synth.sample_rows(w, 10)
     assert len(s) == 10 and s[0] == 0 and s[-1] == w.channels - 1
     assert s == synth.sample_rows(w, 10)
+
+
+def test_nd_workloads_and_kernels():
+    for w in synth.ND_WORKLOADS:
+        assert w.grid == int(np.prod(w.dims))
+        assert w.padded == int(np.prod([2 * d if w.boundary == "zero" else d for d in w.dims]))
+        assert w.padded <= 16384                      # one on-chip grid per (channel, pair)
+        assert w.roofline_bytes() == ((w.N + 2) * w.B * w.D * w.grid * w.elem_bytes
+                                      + w.N * w.D * w.padded * 8)
+    w = synth.nd_custom(2, "f32", 2, 3, (4, 8), "circular", seed=9)
+    K1, K2 = synth.nd_kernels(w), synth.nd_kernels(w)
+    assert K1.shape == (2, 3, 32) and K1.dtype == np.float32
+    np.testing.assert_array_equal(K1, K2)             # seeded, reproducible
+    # the window peaks at offset 0 and, on a circular grid, is symmetric in the periodic distance
+    Kz = synth.nd_kernels(synth.nd_custom(1, "f32", 1, 1, (16,), "circular", seed=1))[0, 0]
+    g = synth.normal(1, 500, 0, 16)
+    win = Kz / g
+    np.testing.assert_allclose(win[1:], win[1:][::-1], rtol=1e-5)
+    assert np.argmax(win) == 0
+    np.testing.assert_allclose(np.linalg.norm(win), 1.0, rtol=1e-5)
+    v, xs = synth.nd_inputs(w)
+    assert v.shape == (6, 32) and len(xs) == 2
