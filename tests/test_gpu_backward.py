@@ -76,11 +76,9 @@ SWEEP = [
     # N, dtype, B, D, L
     (1, "f32", 1, 1, 16),        # zero-extended 128-point grid
     (2, "f32", 2, 3, 64),
-    (2, "f32", 2, 2, 256),
     (3, "f32", 1, 2, 512),
     (2, "bf16", 2, 3, 1024),
     (2, "f32", 3, 2, 2048),
-    (2, "bf16", 1, 3, 4096),
     (3, "bf16", 2, 2, 8192),
     (2, "f32", 1, 2, 16384),     # four-step
     (2, "bf16", 2, 1, 32768),    # four-step
