@@ -191,3 +191,37 @@ def test_nd_queries_and_host_rejections(lib):
     assert g(p, xs, xs, 0, 1, 2, ok, 0, 2, 0, p, None) == hy.HYENA_ERR_INVALID_ARG
     assert g(p, xs, xs, 1, 1, 2, I3(8, 6, 0), 0, 2, 0, p, None) == hy.HYENA_ERR_UNSUPPORTED
     assert g(p, xs, xs, 1, 1, 0, ok, 0, 2, 0, p, None) == hy.HYENA_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
+    """include/hyena.h compiles as strict C99, and a C program linked against
+    the library calls its host-side queries (no device needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    inc = os.path.join(hy._PKG, os.pardir, "include")
+    src = tmp_path / "probe.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "hyena.h"\n'
+        "int main(void) {\n"
+        "  int dims[2] = {64, 64}, M = 0, M1 = 0, MV = 0;\n"
+        "  if (hyena_spectrum_layout(131072, &M, &M1, &MV) != HYENA_OK) return 2;\n"
+        '  printf("%d %zu %zu %zu %d %d %d\\n", hyena_abi_version(), hyena_filter_spectrum_bytes(768, 2048),\n'
+        "         hyena_filter_spectrum_bytes_f16(768, 2048), hyena_nd_spectrum_bytes(4, 2, dims, HYENA_ND_ZERO),\n"
+        "         M, M1, MV);\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "probe"
+    libdir = os.path.dirname(hy.LIB_PATH)
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", f"-I{inc}", str(src), "-o",
+                        str(exe), f"-L{libdir}", "-lhyena_b200", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    I2 = ctypes.c_int * 2
+    assert int(out[0]) == hy.abi_version()
+    assert int(out[1]) == lib.hyena_filter_spectrum_bytes(768, 2048)
+    assert int(out[2]) == lib.hyena_filter_spectrum_bytes_f16(768, 2048)
+    assert int(out[3]) == lib.hyena_nd_spectrum_bytes(4, 2, I2(64, 64), 0)
+    assert tuple(int(t) for t in out[4:7]) == hy.spectrum_layout(131072)
