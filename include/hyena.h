@@ -291,6 +291,9 @@ const char *hyena_last_cuda_error(void);
  *   hG:            device float32 [D][lg], 1 <= lg <= 1024 (SE: a few taps;
  *                  MR: hundreds, e.g. an explicit filter times a decay)
  * Any L >= 1. Arithmetic in float32; bf16 results rounded to nearest even.
+ * Every pointer must be 16-byte aligned. Errors: HYENA_ERR_INVALID_ARG
+ * (alignment, lf, lg, B, D or L out of range, B*D*L above 2^40),
+ * HYENA_ERR_CUDA (launch). Asynchronous on stream.
  */
 hyena_status hyena_striped_forward(const void *xq, const void *xk, const void *xv, const float *hT, const float *hH,
                                    const float *hK, int lf, const float *hG, int lg, int B, int D, int L,
@@ -300,7 +303,8 @@ hyena_status hyena_striped_forward(const void *xq, const void *xk, const void *x
  * The featurizer half of the operator for a long implicit inner filter
  * (Hyena-LI): q = hT * xq and u = (hH * xk) (.) (hK * xv), device [B][D][L]
  * dtype. The operator is then y = hyena_forward(u, {q}, {hyena_filter_rfft(hG)},
- * N = 1). Arguments as in hyena_striped_forward.
+ * N = 1). Arguments, alignment and errors as in hyena_striped_forward; q and u
+ * must not alias the inputs.
  */
 hyena_status hyena_striped_featurize(const void *xq, const void *xk, const void *xv, const float *hT,
                                      const float *hH, const float *hK, int lf, int B, int D, int L,
@@ -310,15 +314,18 @@ hyena_status hyena_striped_featurize(const void *xq, const void *xk, const void 
  * Hyena-LI filter ("02. 3つの Hyena 演算子", section 3): a sum of real
  * exponentials, h[c][t] = sum_{n < d} R[c][n] lambda[c][n]^t for t < L (the
  * page's exponent t - 1 with 1-based t). R, lambda: device float32 [D][d],
- * 1 <= d <= 64; h: device float32 [D][L].
+ * 1 <= d <= 64; h: device float32 [D][L]. Pointers 16-byte aligned.
+ * Errors: HYENA_ERR_INVALID_ARG (alignment, d, D, L), HYENA_ERR_CUDA.
  */
 hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d, int D, int L, float *h,
                                       hyena_stream stream);
 
 /*
- * Kernels that wait on mbarriers for asynchronous tensor-core work (the
- * tcgen05 forward for bf16, L = 2048, B even, in libraries built with
- * HYENA_TC05) bound every wait by an iteration limit; a wait that runs out
+ * Kernels that wait on mbarriers for asynchronous copies or tensor-core work
+ * (the striped bulk-copy kernel of hyena_striped_forward, taken when a row's
+ * byte length is a multiple of 16; the tcgen05 forward for bf16, L = 2048,
+ * B even, in libraries built with HYENA_TC05) bound every wait by an
+ * iteration limit; a wait that runs out
  * makes every thread block of that launch stop early (its outputs are then
  * invalid) and sets a sticky flag on the current device. This call
  * synchronises with the device, reads and clears the flag: HYENA_OK if no
