@@ -19,7 +19,9 @@
  * Conventions for every call:
  *  - Every pointer named "device" is CUDA device memory of the current
  *    device, 16-byte aligned; the caller owns it. The library never
- *    allocates device memory and keeps no state between calls.
+ *    allocates device memory and keeps no state between calls, apart from
+ *    the static scratch of hyena_forward_static_workspace and the sticky
+ *    timeout flag that hyena_device_timeouts reads and clears.
  *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
  *    the legacy default stream). Inputs must stay valid until the work on
  *    the stream has finished.
@@ -29,8 +31,10 @@
  *  - Activations v, x_n, y are row-major [B][D][L] (time fastest) in the
  *    storage type `dtype`; the arithmetic is float32 throughout and bf16
  *    results are rounded to nearest even.
- *  - L must be a power of two with 16 <= L <= 2^20 (HYENA_ERR_UNSUPPORTED
- *    otherwise); 1 <= N <= 8; B, D >= 1.
+ *  - For the 1-D FFT calls L must be a power of two with 16 <= L <= 2^20
+ *    (HYENA_ERR_UNSUPPORTED otherwise); 1 <= N <= 8; B, D >= 1. The
+ *    StripedHyena calls take any L >= 1 and the HyenaND calls state their
+ *    own grid rules.
  *  - All entry points are thread-safe.
  */
 #ifndef HYENA_B200_H
@@ -47,7 +51,7 @@ extern "C" {
 typedef enum {
   HYENA_OK = 0,
   HYENA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad count or dtype */
-  HYENA_ERR_UNSUPPORTED = 2,   /* L not a power of two in [16, 2^20] */
+  HYENA_ERR_UNSUPPORTED = 2,   /* shape outside what the call supports (e.g. L not a power of two in [16, 2^20]) */
   HYENA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
   HYENA_ERR_CUDA = 4,          /* a CUDA launch or attribute call failed */
   HYENA_ERR_TIMEOUT = 5        /* a bounded device-side wait ran out (see hyena_device_timeouts) */
