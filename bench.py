@@ -5,16 +5,20 @@
                     [--pass forward|backward]
 
 A step is one hyena_forward over one batch of the workload (default: the
-order-2, bf16, B=4, D=768, L=2048 workload), with the filter spectra already
-cached (they depend only on the weights). Inputs are resident in HBM when the
+largest one-GPU workload, order 2, bf16, B=1, D=256, L=2^20), with the filter
+spectra already cached (they depend only on the weights; filter generation
+and the spectrum are timed on their own and reported beside the line, not in
+it). Inputs are resident in HBM when the
 timed region starts and are rotated over enough buffer sets that the step's
 working set is not in L2. The metric is B*D*L processed per second (x1e9)
 and the fraction of the HBM roofline; one JSON line is printed by rank 0.
 
 --gpus N > 1 runs under torchrun: every rank processes its own batch
 (weak scaling, no collective on the data path); time is the max over ranks.
---impl reference times the float64 CPU oracle on a bounded sample of the
-same workload (rank 0 only).
+--impl reference times the float64 CPU oracle (rank 0 only): every one of
+its W warm-up and K timed steps is one pass of the oracle over the same
+bounded sample of rows of the workload, sized so the whole run takes a few
+minutes; its config is the one the GPU arm prints.
 The e2e figure times steps through the public API with every step's inputs
 copied in from pinned host memory and its result copied back; forward,
 striped and ND steps rotate over three CUDA streams so that one step's
@@ -71,14 +75,7 @@ KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "tc": ("tc_fused.cu", "fft_engine.cuh", "layout.h"),
-    "tc05": ("tc05.cu", "fft_engine.cuh", "kernels.cuh", "layout.h"),
 }
-
-
-def tc05_built() -> bool:
-    """True when the library was built with the tcgen05 forward (build.py --tc05)."""
-    from fft_long_convolution_implicit_b200 import build as hybuild
-    return hybuild.built_tc05()
 
 
 def dominant_kernel(w: synth.Workload, spec16: bool = False) -> tuple[str, str]:
@@ -87,8 +84,6 @@ def dominant_kernel(w: synth.Workload, spec16: bool = False) -> tuple[str, str]:
         return "four-step column/row kernels (whole step)", "fourstep"
     if spec16:
         return "fused_forward_kernel (f16 spectra)", "fused"
-    if w.dtype == "bf16" and w.B % 2 == 0 and w.L == 2048 and tc05_built():
-        return "tc05_forward_kernel", "tc05"
     if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
         return "tc_forward_kernel", "tc"
     return "fused_forward_kernel", "fused"
@@ -270,6 +265,54 @@ def oracle_sample(w: synth.Workload, target_core_seconds: float = 12.0, backward
             "seconds": dt}
 
 
+def oracle_passes(w: synth.Workload, steps: int, warmup: int, backward: bool = False,
+                  striped: bool = False, budget_s: float = 120.0):
+    """Reference arm: `warmup` untimed and `steps` timed passes of the float64
+    oracle (as it stands) over one bounded sample of rows of the workload,
+    one row per host core at least; every pass recomputes the whole sample.
+    The sample is sized so that all passes take about budget_s seconds of
+    wall time. Returns (seconds of each timed pass, rows per pass, cores)."""
+    import oracle
+    threads = host_cores()
+    if striped:
+        hT, hH, hK, hG = synth.striped_filters(w, STRIPED_LF, STRIPED_LG)
+    else:
+        wt = synth.filter_weights(w)
+
+    def prepare(rows):
+        if striped:
+            xv, (xq, xk) = synth.inputs(synth.Workload(**{**w.__dict__, "N": 2}), rows)
+            fr = [r % w.D for r in rows]
+            return lambda n_threads: oracle.striped_forward(xq, xk, xv, hT, hH, hK, hG, filter_row=fr,
+                                                            threads=n_threads)
+        v, xs = synth.inputs(w, rows)
+        cs = sorted({r % w.D for r in rows})
+        hrows = oracle.implicit_filter(wt, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi,
+                                       rows=[(n, c) for n in range(w.N) for c in cs], threads=threads)
+        hs = [hrows[n * len(cs):(n + 1) * len(cs)] for n in range(w.N)]
+        fr = [cs.index(r % w.D) for r in rows]
+        dy = synth.dy_rows(w, rows) if backward else None
+        if backward:
+            return lambda n_threads: oracle.hyena_backward(v, xs, hs, dy, filter_row=fr, threads=n_threads)
+        return lambda n_threads: oracle.hyena_forward(v, xs, hs, filter_row=fr, threads=n_threads)
+
+    one = prepare([0])
+    t0 = time.perf_counter()
+    one(1)
+    per_row = max(time.perf_counter() - t0, 1e-5)
+    per_pass = max(per_row, budget_s / max(1, steps + warmup))
+    nrows = int(min(w.channels, threads * max(1, int(per_pass / per_row))))
+    run = prepare(list(range(nrows)))
+    for _ in range(warmup):
+        run(threads)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        run(threads)
+        times.append(time.perf_counter() - t0)
+    return times, nrows, threads
+
+
 def oracle_striped_sample(w: synth.Workload, target_core_seconds: float = 8.0):
     """The float64 StripedHyena-form oracle on a bounded sample of rows."""
     import oracle
@@ -357,23 +400,67 @@ def oracle_nd_sample(w: "synth.NDWorkload", target_core_seconds: float = 8.0):
                       f"({w.boundary} boundary)", "seconds": dt}
 
 
+def nd_rotation(w: "synth.NDWorkload") -> tuple[int, int]:
+    """(bytes of one ND input set, number of sets rotated over): the step's algorithmic bytes set the size."""
+    set_bytes = w.roofline_bytes()
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    return set_bytes, nsets
+
+
+def nd_config(w: "synth.NDWorkload", world: int) -> dict:
+    """The config dict both arms print for an ND workload."""
+    set_bytes, nsets = nd_rotation(w)
+    return {"workload": w.name, "B": w.B, "D": w.D, "dims": list(w.dims), "boundary": w.boundary, "N": w.N,
+            "io": w.dtype, "pass": "nd", "global_batch": w.B * world, "parallelism": f"replicas x{world}",
+            "l2": (f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
+                   f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)") if nsets > 1 else
+                  f"inputs of {set_bytes / 2**20:.0f} MiB per step, larger than L2"}
+
+
 def run_nd(args) -> int:
     w = synth.nd_workload(args.nd_config)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = {"workload": w.name, "B": w.B, "D": w.D, "dims": list(w.dims), "boundary": w.boundary, "N": w.N,
-           "io": w.dtype, "pass": "nd"}
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_nd_sample(w)
-        print(json.dumps({"impl": "reference", "metric": METRIC_ND, "value": cb["value"], "unit": UNIT_ND,
+        import oracle
+        K = synth.nd_kernels(w)
+
+        def prepare(rows):
+            v, xs = synth.nd_inputs(w, rows)
+            fr = [r % w.D for r in rows]
+            return lambda: oracle.hyena_nd_forward(v, xs, [K[n] for n in range(w.N)], w.dims, w.boundary,
+                                                   filter_row=fr)
+
+        one = prepare([0])
+        t0 = time.perf_counter()
+        one()
+        per_row = max(time.perf_counter() - t0, 1e-5)
+        per_pass = max(per_row, 120.0 / max(1, args.steps + args.warmup))
+        nrows = int(min(w.channels, max(1, int(per_pass / per_row))))
+        run = prepare(list(range(nrows)))
+        for _ in range(args.warmup):
+            run()
+        times = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            run()
+            times.append(time.perf_counter() - t0)
+        mean_s = statistics.mean(times)
+        value = nrows * w.grid / mean_s / 1e9
+        sample = (f"each of the {args.steps} timed steps (after {args.warmup} warm-up steps) is one oracle pass over "
+                  f"the same {nrows} of {w.channels} (b,c) rows of {w.name}, all N={w.N} stages, numpy FFT "
+                  f"({w.boundary} boundary), one thread")
+        print(json.dumps({"impl": "reference", "metric": METRIC_ND, "value": value, "unit": UNIT_ND,
                           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                          "ms_per_step": w.channels * w.grid / (cb["value"] * 1e9) * 1e3, "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
-                          "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
-                          "e2e": {"value": cb["value"], "unit": UNIT_ND, "h2d_bytes_per_step": 0,
+                          "ms_per_step": mean_s * 1e3, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": nd_config(w, world),
+                          "cpu_baseline": {"value": value, "unit": UNIT_ND, "cores": 1, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": value, "unit": UNIT_ND, "h2d_bytes_per_step": 0,
                                   "d2h_bytes_per_step": 0}}))
         return 0
 
@@ -402,8 +489,7 @@ def run_nd(args) -> int:
     base_v = torch.from_numpy(v_np).view(w.B, w.D, w.grid).to(dev).to(dt)
     base_x = [torch.from_numpy(x).view(w.B, w.D, w.grid).to(dev).to(dt) for x in xs_np]
     base_k = [hy.nd_filter_spectrum(torch.from_numpy(K[n]).to(dev), w.dims, w.boundary) for n in range(w.N)]
-    set_bytes = (w.N + 2) * w.channels * w.grid * w.elem_bytes + sum(t.numel() for t in base_k)
-    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    set_bytes, nsets = nd_rotation(w)
     sets = []
     for i in range(nsets):
         if i == 0:
@@ -454,6 +540,8 @@ def run_nd(args) -> int:
         call = hy.PreparedND(dv, dxs, base_k, w.dims, w.boundary, stream=st)
         return [dv, *dxs], lambda: [call()], [torch.empty_like(pinned_in[0]).pin_memory()]
 
+    if args.e2e_steps is None:
+        args.e2e_steps = int(min(200, max(5, 4e9 // ((w.N + 2) * w.channels * w.grid * w.elem_bytes))))
     e2e_ms = pipelined_e2e(torch, dev, stream, pinned_in, nd_slot, args.e2e_steps, world, dist)
     e2e_value = whole_job_throughput(args.e2e_steps * w.channels * w.grid, world, e2e_ms)
     line = None
@@ -462,9 +550,7 @@ def run_nd(args) -> int:
             "metric": METRIC_ND, "value": round(value, 4), "unit": UNIT_ND, "n_gpus": world, "steps": K_steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K_steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {**cfg, "global_batch": w.B * world, "parallelism": f"replicas x{world}",
-                       "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
-                             f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
+            "config": nd_config(w, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
                          "alg_bytes_per_launch": alg_bytes, "kernel": "nd_forward_kernel",
@@ -490,6 +576,76 @@ def run_nd(args) -> int:
     return 0
 
 
+# ------------------------------------------------------ shared config --
+
+def rotation(w: synth.Workload, which: str) -> tuple[int, int]:
+    """(bytes of one input set, number of sets) the timed steps rotate over
+    so that a set is not in L2 when it is reused: the step's algorithmic
+    bytes (activations and spectra) set the size."""
+    if which == "striped":
+        set_bytes = 4 * w.channels * w.L * w.elem_bytes
+    else:
+        set_bytes = w.roofline_bytes() + (w.channels * w.L * w.elem_bytes if which == "backward" else 0)
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    return set_bytes, nsets
+
+
+def run_config(w: synth.Workload, which: str, spec16: bool, world: int) -> dict:
+    """The config dict both arms print for a workload."""
+    set_bytes, nsets = rotation(w, which)
+    if nsets > 1:
+        l2 = (f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
+              f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)")
+    else:
+        l2 = f"inputs of {set_bytes / 2**20:.0f} MiB per step, larger than L2 ({L2_BYTES / 2**20:.0f} MiB)"
+    return {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype, "pass": which,
+            "spectra": "f16" if spec16 else "f32", "global_batch": w.B * world,
+            "parallelism": f"replicas x{world}", "l2": l2}
+
+
+def filter_timings(torch, hy, tw, h, specs, w: synth.Workload, stream, reps: int = 3) -> dict:
+    """CUDA-event times of hyena_filter_generate (all N filters) and of
+    hyena_filter_rfft (all N spectra) on the step's stream, best of `reps`
+    after one warm-up call each. They run once per weights, so they are
+    reported beside the line and not counted in its value."""
+    def best(fn):
+        fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            out.append(a.elapsed_time(b))
+        return min(out)
+
+    gen_ms = best(lambda: hy.filter_generate(tw, w.N, w.D, w.L, w.alpha_lo, w.alpha_hi, h=h, stream=stream))
+    rfft_ms = best(lambda: [hy.filter_rfft(h[n], hhat=specs[n], stream=stream) for n in range(w.N)])
+    flops = filter_gen_flops(w)
+    peak_tf = None
+    try:
+        with open(PEAKS_FILE) as f:
+            peak_tf = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        pass
+    gen_tf = flops / (gen_ms * 1e-3) / 1e12
+    return {"excluded_from_value": True, "generate_ms": round(gen_ms, 4), "rfft_ms": round(rfft_ms, 4),
+            "generate_flops": flops, "generate_tflops": round(gen_tf, 2),
+            "generate_frac_of_bf16_peak": round(gen_tf / peak_tf, 4) if peak_tf else None,
+            "generate_arithmetic": "float32 SIMT (CUDA cores)",
+            "rfft_bytes": w.N * w.D * w.L * 4 + w.N * w.D * (w.L + 1) * 8}
+
+
+def filter_gen_flops(w: synth.Workload) -> int:
+    """Multiply-add flops of the implicit-filter FFN over all L taps: two
+    hidden layers of width `width` and the output layer of N*D."""
+    e = 1 + 2 * w.n_bands
+    return 2 * w.L * (e * w.width + w.width * w.width + w.width * w.N * w.D)
+
+
 # ---------------------------------------------------------------- main --
 
 def main():
@@ -498,8 +654,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=1, help="workload index (default 1: B=4 D=768 L=2048 N=2 bf16)")
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--config", type=int, default=4,
+                    help="workload index (default 4: the largest one-GPU workload, B=1 D=256 L=2^20 N=2 bf16)")
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="end-to-end steps (default: enough for about 4 GB of host copies, 5 to 200)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="which", choices=["forward", "backward", "striped", "nd"], default="forward")
     ap.add_argument("--nd-config", type=int, default=1, help="HyenaND workload index for --pass nd")
@@ -527,17 +685,24 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    spec16 = args.spectrum == "f16" and args.which == "forward"
     if args.impl == "reference":
         if rank != 0:
             return 0
-        cb = oracle_striped_sample(w) if striped else oracle_sample(w, backward=bwd)
-        line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": UNIT, "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.channels * w.L / (cb["value"] * 1e9) * 1e3,
+        times, nrows, cores = oracle_passes(w, args.steps, args.warmup, backward=bwd, striped=striped)
+        mean_s = statistics.mean(times)
+        value = nrows * w.L / mean_s / 1e9
+        what = ("StripedHyena-SE (lf=%d, lg=%d), direct FIR sums" % (STRIPED_LF, STRIPED_LG) if striped else
+                ("backward (forward again, then gradients)" if bwd else "forward") + f", all N={w.N} stages, " +
+                ("direct O(L^2)" if w.L <= 8192 else "radix-2 FFT") + " causal sums, filters precomputed")
+        sample = (f"each of the {args.steps} timed steps (after {args.warmup} warm-up steps) is one oracle pass "
+                  f"over the same {nrows} of {w.channels} (b,c) rows of {w.name}: {what}")
+        line = {"impl": "reference", "metric": metric, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N,
-                                                 "io": w.dtype, "pass": args.which},
-                "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
-                "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "data": "synthetic", "config": run_config(w, args.which, spec16, world),
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return 0
 
@@ -572,16 +737,13 @@ def main():
     base_v = torch.from_numpy(v_np).view(w.B, w.D, w.L).to(dev).to(dt)
     base_x = [torch.from_numpy(x).view(w.B, w.D, w.L).to(dev).to(dt) for x in xs_np]
     base_h = [hy.filter_rfft(h[n]) for n in range(w.N)]
-    spec16 = args.spectrum == "f16" and args.which == "forward"
+    # filter generation and the spectrum (once per weights): timed on their own, outside the line's value
+    filters = filter_timings(torch, hy, tw, h, base_h, w, stream)
     if spec16:
         base_h = [hy.spectrum_to_f16(t, w.D, w.L) for t in base_h]
     del h
     base_dy = (torch.from_numpy(synth.dy_rows(wr)).view(w.B, w.D, w.L).to(dev).to(dt) if bwd else None)
-    set_bytes = ((w.N + 2 + (1 if bwd else 0)) * w.channels * w.L * w.elem_bytes
-                 + sum(t.numel() for t in base_h))
-    if striped:
-        set_bytes = 3 * w.channels * w.L * w.elem_bytes
-    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes)) if set_bytes < 3 * L2_BYTES else 1
+    set_bytes, nsets = rotation(w, args.which)
     shared_out = None
     if bwd:
         # one set of outputs and one workspace, shared by every input set
@@ -655,6 +817,9 @@ def main():
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
 
     # end to end through the public API: pinned host inputs in, result out
+    if args.e2e_steps is None:
+        copy_bytes = (w.N + 2 + (2 * w.N + 2 if bwd else 0)) * w.channels * w.L * w.elem_bytes
+        args.e2e_steps = int(min(200, max(5, 4e9 // copy_bytes)))
     pin_v = base_v.cpu().pin_memory()
     pin_x = [x.cpu().pin_memory() for x in base_x]
     dv = torch.empty_like(base_v)
@@ -721,11 +886,7 @@ def main():
             "metric": metric, "value": round(value, 4), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "D": w.D, "L": w.L, "N": w.N, "io": w.dtype, "pass": args.which,
-                       "spectra": "f16" if spec16 else "f32",
-                       "global_batch": w.B * world, "parallelism": f"replicas x{world}",
-                       "l2": f"inputs rotated over {nsets} buffer sets of {set_bytes / 2**20:.0f} MiB "
-                             f"(> L2 {L2_BYTES / 2**20:.0f} MiB between reuses)"},
+            "config": run_config(w, args.which, spec16, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "traffic": None if (bwd or striped or spec16) else measured_traffic(w.name),
@@ -739,6 +900,8 @@ def main():
             "gpu_launches": K * launches_per_step,
             "clocks": clocks,
         }
+        if not striped:
+            line["filters"] = filters
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -1,12 +1,6 @@
 """Build the sm_100a shared library libhyena_b200.so in-tree.
 
-    python -m fft_long_convolution_implicit_b200.build [--force] [--verbose-ptxas] [--tc05]
-
---tc05 builds the variant whose bf16, L = 2048 forward runs on the tcgen05
-kernel (csrc/tc05.cu) instead of the mma.sync one (-DHYENA_TC05=1); the
-choice is remembered in lib/build_options.txt; build() called without a
-variant (as the tests and bench.py do) keeps the recorded one, and
-`python -m ...build` without --tc05 builds the default.
+    python -m fft_long_convolution_implicit_b200.build [--force] [--verbose-ptxas]
 
 Each csrc/*.cu is compiled separately (in parallel) with
 ``-gencode arch=compute_100a,code=sm_100a -lineinfo`` and linked into
@@ -53,43 +47,34 @@ def _deps():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def _defines(tc05: bool) -> list[str]:
-    return ["-DHYENA_TC05=1"] if tc05 else []
+def _objects_stale() -> bool:
+    """An object file whose source is gone (a removed kernel) must not be linked."""
+    srcs = {os.path.basename(s) + ".o" for s in _sources()}
+    return any(os.path.basename(o) not in srcs for o in glob.glob(os.path.join(OBJ, "*.o")))
 
 
-def up_to_date(tc05: bool = False) -> bool:
-    if not os.path.exists(LIB) or not os.path.exists(OPTIONS):
+def up_to_date() -> bool:
+    if not os.path.exists(LIB) or not os.path.exists(OPTIONS) or _objects_stale():
         return False
-    with open(OPTIONS) as f:
-        if f.read().strip() != " ".join(_defines(tc05)):
-            return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(d) <= t for d in _deps() + [__file__])
 
 
-def built_tc05() -> bool:
-    """The variant recorded by the last build (False when none is recorded)."""
-    try:
-        with open(OPTIONS) as f:
-            return "HYENA_TC05=1" in f.read()
-    except OSError:
-        return False
-
-
-def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True, tc05: bool | None = None) -> str:
-    """tc05=None keeps the variant of the last build (the default one if none)."""
-    if tc05 is None:
-        tc05 = built_tc05()
-    if not force and up_to_date(tc05):
+def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True) -> str:
+    if not force and up_to_date():
         return LIB
     os.makedirs(OBJ, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
+    srcs_o = {os.path.basename(s) + ".o" for s in _sources()}
+    for o in glob.glob(os.path.join(OBJ, "*.o")):
+        if os.path.basename(o) not in srcs_o:
+            os.remove(o)
     cc = nvcc()
     srcs = _sources()
 
     def compile_one(src):
         obj = os.path.join(OBJ, os.path.basename(src) + ".o")
-        cmd = [cc, *ARCH, *FLAGS, *_defines(tc05), "-c", src, "-o", obj]
+        cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
         if verbose_ptxas:
             cmd += ["-Xptxas", "-v"]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -109,7 +94,7 @@ def build(force: bool = False, verbose_ptxas: bool = False, quiet: bool = True, 
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
     with open(OPTIONS, "w") as f:
-        f.write(" ".join(_defines(tc05)) + "\n")
+        f.write("default\n")
     if not quiet:
         print(f"built {LIB}")
     return LIB
@@ -119,6 +104,5 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
-    ap.add_argument("--tc05", action="store_true", help="bf16 L=2048 forward on the tcgen05 kernel")
     a = ap.parse_args()
-    build(force=a.force, verbose_ptxas=a.verbose_ptxas, quiet=False, tc05=bool(a.tc05))
+    build(force=a.force, verbose_ptxas=a.verbose_ptxas, quiet=False)

@@ -21,13 +21,6 @@ hyena_status cuda_fail(cudaError_t e) {
 
 bool aligned16(const void* p) { return p && ((reinterpret_cast<uintptr_t>(p) & 15u) == 0); }
 
-// L = 2048 bf16 pairs: tcgen05 kernel (tc05.cu) when built with HYENA_TC05=1,
-// otherwise the mma.sync kernel (tc_fused.cu)
-#ifndef HYENA_TC05
-#define HYENA_TC05 0
-#endif
-constexpr bool kUseTc05 = HYENA_TC05 != 0;
-
 // L2-sized wave of four-step channels
 constexpr size_t kWaveTargetBytes = size_t(48) << 20;
 constexpr long long kMaxGridY = 65535;
@@ -106,7 +99,7 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
       // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
       for (int n = 0; n < N; ++n)
         p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
-      e = (kUseTc05 && ly.R0 == 16) ? launch_tc05_forward(p, s) : launch_tc_forward(p, ly, s);
+      e = launch_tc_forward(p, ly, s);
     } else {
       e = launch_fused_forward(p, ly.logMV, s);
     }
@@ -155,8 +148,7 @@ cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, con
   if (!ly.fourstep) {
     e = launch_fused_spectrum(h, spec, tables, rows, ly.L, ly.logMV, s);
     if (e == cudaSuccess && with_tc && ly.tc)
-      e = (kUseTc05 && ly.R0 == 16) ? launch_tc05_spectrum(spec, spec + tc_spectrum_offset(ly, rows), rows, ly.M, s)
-                                    : launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
+      e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
   } else {
     for (long long c0 = 0; c0 < rows && e == cudaSuccess; c0 += kMaxGridY) {
       const int nd = (int)((rows - c0) < kMaxGridY ? (rows - c0) : kMaxGridY);
@@ -185,10 +177,9 @@ const char* hyena_status_string(hyena_status s) {
 const char* hyena_last_cuda_error(void) { return g_last_cuda_error; }
 
 hyena_status hyena_device_timeouts(void) {
-  const int a = tc05_read_and_clear_timeout();
   const int b = striped_read_and_clear_timeout();
-  if (a < 0 || b < 0) return cuda_fail(cudaGetLastError());
-  return (a || b) ? HYENA_ERR_TIMEOUT : HYENA_OK;
+  if (b < 0) return cuda_fail(cudaGetLastError());
+  return b ? HYENA_ERR_TIMEOUT : HYENA_OK;
 }
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {
@@ -274,6 +265,9 @@ hyena_status hyena_forward_f16_spectra(const void* v, const void* const* x, cons
                                        size_t workspace_bytes, hyena_stream stream) {
   if (N < 1 || N > kMaxOrder || B < 1 || D < 1) return HYENA_ERR_INVALID_ARG;
   if (dtype != HYENA_F32 && dtype != HYENA_BF16) return HYENA_ERR_INVALID_ARG;
+  // f16 bins carry a relative rounding of 2^-11 per stage, far above what
+  // float32 I/O promises; only bf16 I/O (whose own rounding is 2^-9) is served
+  if (dtype != HYENA_BF16) return HYENA_ERR_UNSUPPORTED;
   if (!x || !hhat16 || !aligned16(v) || !aligned16(y)) return HYENA_ERR_INVALID_ARG;
   for (int n = 0; n < N; ++n)
     if (!aligned16(x[n]) || !aligned16(hhat16[n])) return HYENA_ERR_INVALID_ARG;

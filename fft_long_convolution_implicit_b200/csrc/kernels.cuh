@@ -86,11 +86,6 @@ cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* ta
 cudaError_t launch_tc_forward(const FusedLaunch& p, const Layout& y, cudaStream_t s);
 cudaError_t launch_tc_spectrum(const float2* nat, float2* tcs, float2* tables, int D, const Layout& y,
                                cudaStream_t s);
-// tcgen05 forward and its spectrum copy (L = 2048); the sticky timeout flag of
-// its bounded mbarrier waits (-1 if it cannot be read).
-cudaError_t launch_tc05_forward(const FusedLaunch& p, cudaStream_t s);
-cudaError_t launch_tc05_spectrum(const float2* nat, float2* tcs, int D, int M, cudaStream_t s);
-int tc05_read_and_clear_timeout();
 // StripedHyena-form operator: featurizer length <= kMaxStripedLF, explicit
 // inner filter length <= kMaxStripedLG. hG == nullptr: featurize only (q, u).
 constexpr int kMaxStripedLF = 16;

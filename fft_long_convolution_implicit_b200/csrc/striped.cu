@@ -225,18 +225,31 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
-__device__ __forceinline__ bool st_mbar_wait(uint32_t bar, uint32_t phase) {
-  for (int it = 0; it < (1 << 24); ++it) {
+__device__ __forceinline__ unsigned long long st_globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase of an mbarrier to complete, bounded in time: each
+// try_wait suspends for at most kStTrySuspendNs, and the wait gives up once
+// kStWaitLimitNs of global time have passed since it started (returns false).
+constexpr unsigned kStTrySuspendNs = 20000;                 // 20 us per try
+constexpr unsigned long long kStWaitLimitNs = 200000000ull; // 0.2 s per wait
+__device__ __forceinline__ bool st_mbar_wait(uint32_t bar, uint32_t phase,
+                                             unsigned long long limit_ns = kStWaitLimitNs) {
+  const unsigned long long t0 = st_globaltimer_ns();
+  for (;;) {
     uint32_t done;
     asm volatile(
-        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, P1;\n\t}\n"
         : "=r"(done)
-        : "r"(bar), "r"(phase)
+        : "r"(bar), "r"(phase), "r"(kStTrySuspendNs)
         : "memory");
     if (done) return true;
+    if (st_globaltimer_ns() - t0 > limit_ns) return false;
   }
-  return false;
 }
 
 template <typename T>
@@ -442,11 +455,11 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
   }
-  // after a timeout: wait (bounded) for the copies still in flight into this
-  // CTA's shared memory before it exits (normal exits leave none)
+  // after a timeout: wait (bounded, 1 s each) for the copies still in flight
+  // into this CTA's shared memory before it exits (normal exits leave none)
   if (tid == 0)
     for (int k = 0; k < 2; ++k)
-      if (pending[k]) st_mbar_wait(st_smem_u32(&bars[k]), phase[k]);
+      if (pending[k]) st_mbar_wait(st_smem_u32(&bars[k]), phase[k], 1000000000ull);
   __syncthreads();
 }
 

@@ -35,7 +35,9 @@
  *    (HYENA_ERR_UNSUPPORTED otherwise); 1 <= N <= 8; B, D >= 1. The
  *    StripedHyena calls take any L >= 1 and the HyenaND calls state their
  *    own grid rules.
- *  - All entry points are thread-safe.
+ *  - All entry points may be called from several host threads at once, with
+ *    one exception: calls of hyena_forward_static_workspace share one device
+ *    scratch array, so two of them whose GPU work overlaps race (see there).
  */
 #ifndef HYENA_B200_H
 #define HYENA_B200_H
@@ -148,9 +150,13 @@ hyena_status hyena_forward(const void *v, const void *const *x, const void *cons
  * behind its back, fixed-budget deployments, and latency-critical paths that
  * cannot afford cudaMalloc's implicit device synchronisation. This entry point
  * needs no workspace argument: the four-step scratch lives in a file-scope
- * device array of HYENA_STATIC_WORKSPACE_BYTES inside the library, reserved
- * on every GPU that loads the library and held until the process exits.
- * It allocates nothing and calls no allocating routine.
+ * device array of HYENA_STATIC_WORKSPACE_BYTES inside the library. It
+ * allocates nothing and calls no allocating routine itself; the array is
+ * reserved when the library module that holds it is loaded into a CUDA
+ * context -- with CUDA's default lazy module loading, that is the first call
+ * of this entry point in the context (make one warm-up call outside any
+ * phase that must not reserve memory) -- and held until the process exits.
+ * A call rejected by the host-side checks loads nothing.
  *
  *  - Only for 8192 < L <= 2^20 (the lengths whose forward needs scratch);
  *    shorter L returns HYENA_ERR_UNSUPPORTED: use hyena_forward with a NULL
@@ -158,9 +164,11 @@ hyena_status hyena_forward(const void *v, const void *const *x, const void *cons
  *  - Channels are processed in waves of HYENA_STATIC_WORKSPACE_BYTES / (8 L);
  *    a length whose single channel would not fit is rejected with
  *    HYENA_ERR_WORKSPACE (never the case for supported L).
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture on the device.
+ *  - The first call in a CUDA context looks up the array's device address
+ *    (cudaGetSymbolAddress) with that context current and caches it under
+ *    the context's unique id; make that first call before any stream capture
+ *    in the context. A context destroyed and re-created (cudaDeviceReset, or
+ *    a different context made current) is looked up afresh.
  *  - Every call on a device shares the one array and leaves its last
  *    contents there (nothing needs clearing: every element is written before
  *    it is read). Calls whose GPU work overlaps -- on different streams, or
@@ -207,12 +215,13 @@ hyena_status hyena_filter_spectrum_to_f16(const void *hhat, int D, int L, void *
 
 /*
  * hyena_forward_f16_spectra -- hyena_forward whose hhat[n] are f16 blocks
- * from hyena_filter_spectrum_to_f16. Arguments, layouts, aliasing,
- * workspace and errors are those of hyena_forward. It always runs the SIMT
- * kernels (the tensor-core forward reads a float32 copy of its own). The
- * result differs from hyena_forward by the f16 rounding of the spectra:
- * relative L2 about 2^-11 per stage for spectra whose bins span a modest
- * range.
+ * from hyena_filter_spectrum_to_f16, for bf16 I/O only: dtype HYENA_F32
+ * returns HYENA_ERR_UNSUPPORTED, because the f16 rounding of the spectra
+ * (relative L2 up to 2^-11 per stage) is far above the float32 accuracy
+ * that f32 I/O stands for, while it stays below the bf16 output rounding
+ * (2^-9). Other arguments, layouts, aliasing, workspace and errors are those
+ * of hyena_forward. It always runs the SIMT kernels (the tensor-core
+ * forward reads a float32 copy of its own).
  */
 hyena_status hyena_forward_f16_spectra(const void *v, const void *const *x, const void *const *hhat16, int B, int D,
                                        int L, int N, hyena_dtype dtype, void *y, void *workspace,
@@ -325,16 +334,16 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
                                       hyena_stream stream);
 
 /*
- * Kernels that wait on mbarriers for asynchronous copies or tensor-core work
- * (the striped bulk-copy kernel of hyena_striped_forward, taken when a row's
- * byte length is a multiple of 16; the tcgen05 forward for bf16, L = 2048,
- * B even, in libraries built with HYENA_TC05) bound every wait by an
- * iteration limit; a wait that runs out
- * makes every thread block of that launch stop early (its outputs are then
- * invalid) and sets a sticky flag on the current device. This call
- * synchronises with the device, reads and clears the flag: HYENA_OK if no
- * wait ran out since the last call, HYENA_ERR_TIMEOUT otherwise
- * (HYENA_ERR_CUDA if it cannot be read).
+ * Kernels that wait on mbarriers for asynchronous copies (the striped
+ * bulk-copy kernel of hyena_striped_forward, taken when a row's byte length
+ * is a multiple of 16) bound every wait in time: a wait gives up 0.2 s of
+ * GPU global time after it started (each polling step suspends for at most
+ * 20 us). A wait that runs out makes every thread block of that launch stop
+ * early (its outputs are then invalid) and sets a sticky flag on the current
+ * device; before exiting, such a block waits at most 1 s more for the copies
+ * it still has in flight. This call synchronises with the device, reads and
+ * clears the flag: HYENA_OK if no wait ran out since the last call,
+ * HYENA_ERR_TIMEOUT otherwise (HYENA_ERR_CUDA if it cannot be read).
  */
 hyena_status hyena_device_timeouts(void);
 

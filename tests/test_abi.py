@@ -157,11 +157,14 @@ def test_f16_spectra_queries_and_host_rejections(lib):
     assert lib.hyena_filter_spectrum_to_f16(p, 4, 1000, p, None) == hy.HYENA_ERR_UNSUPPORTED
     f = lib.hyena_forward_f16_spectra
     xs = (ctypes.c_void_p * 2)(p, p)
-    assert f(p, xs, xs, 1, 1, 1024, 0, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1024, 0, 1, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
     assert f(p, xs, xs, 1, 1, 1024, 2, 7, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
-    assert f(mis, xs, xs, 1, 1, 1024, 2, 0, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
-    assert f(p, xs, xs, 1, 1, 1000, 2, 0, p, None, 0, None) == hy.HYENA_ERR_UNSUPPORTED
-    assert f(p, xs, xs, 1, 1, 32768, 2, 0, p, None, 0, None) == hy.HYENA_ERR_WORKSPACE
+    assert f(mis, xs, xs, 1, 1, 1024, 2, 1, p, None, 0, None) == hy.HYENA_ERR_INVALID_ARG
+    assert f(p, xs, xs, 1, 1, 1000, 2, 1, p, None, 0, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert f(p, xs, xs, 1, 1, 32768, 2, 1, p, None, 0, None) == hy.HYENA_ERR_WORKSPACE
+    # float32 I/O is refused: f16 spectra cannot meet the float32 accuracy
+    assert f(p, xs, xs, 1, 1, 1024, 2, hy.HYENA_F32, p, None, 0, None) == hy.HYENA_ERR_UNSUPPORTED
+    assert f(p, xs, xs, 1, 1, 32768, 2, hy.HYENA_F32, p, p, 1 << 20, None) == hy.HYENA_ERR_UNSUPPORTED
 
 
 def test_nd_queries_and_host_rejections(lib):

@@ -5,7 +5,13 @@ library's own static device scratch instead of a caller workspace.
 
 Checked through the C ABI against hyena_forward with a caller workspace, on
 two calls in a row (the scratch keeps the previous call's contents, which
-must not leak into the next result). This file is collected last.
+must not leak into the next result): the results are bit for bit equal (the
+two calls differ only in how many channels a wave holds, and every channel's
+arithmetic is the same whatever the wave), one row is checked against the
+float64 oracle, and the device's free memory is the same before and after a
+call (nothing is allocated). The shapes include L = 2^20, where the 16 MiB
+scratch holds two channels per wave and the last wave is partial. This file
+is collected last.
 """
 import ctypes
 
@@ -13,13 +19,13 @@ import numpy as np
 import pytest
 
 import synth
-from hyena_cases import TOL, rel_l2_rows, upload, weights_to_cuda
+from hyena_cases import TOL, oracle_rows, rel_l2_rows, upload, weights_to_cuda
 
 pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("N,dtype,B,D,L", [(2, "bf16", 2, 3, 32768), (2, "bf16", 1, 40, 131072),
-                                           (3, "f32", 1, 2, 16384)])
+                                           (3, "f32", 1, 2, 16384), (2, "bf16", 1, 3, 1 << 20)])
 def test_static_workspace_matches_workspace_forward(N, dtype, B, D, L):
     import torch
     from fft_long_convolution_implicit_b200 import build
@@ -36,22 +42,38 @@ def test_static_workspace_matches_workspace_forward(N, dtype, B, D, L):
     txs = [upload(x, w) for x in xs]
     y_ref = hy.forward(tv, txs, hh)          # caller-provided workspace
     torch.cuda.synchronize()
-    ref = y_ref.double().cpu().numpy().reshape(w.channels, L)
+    ref_bits = y_ref.view(torch.int16 if dtype == "bf16" else torch.int32).cpu().numpy()
 
     code = hy.HYENA_BF16 if dtype == "bf16" else hy.HYENA_F32
     xarr = (ctypes.c_void_p * N)(*[x.data_ptr() for x in txs])
     harr = (ctypes.c_void_p * N)(*[t.data_ptr() for t in hh])
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    ys = [torch.full_like(tv, float("nan")) for _ in range(2)]
+    # a warm-up call loads the library module that holds the scratch
+    assert lib.hyena_forward_static_workspace(ctypes.c_void_p(tv.data_ptr()), xarr, harr, B, D, L, N, code,
+                                              ctypes.c_void_p(ys[0].data_ptr()), stream) == hy.HYENA_OK
+    torch.cuda.synchronize()
     for call in range(2):
-        y = torch.full_like(tv, float("nan"))
+        y = ys[call]
+        y.fill_(float("nan"))
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
+        reserved_before = torch.cuda.memory_reserved()
         st = lib.hyena_forward_static_workspace(ctypes.c_void_p(tv.data_ptr()), xarr, harr, B, D, L, N, code,
                                                 ctypes.c_void_p(y.data_ptr()), stream)
         assert st == hy.HYENA_OK, lib.hyena_status_string(st)
         torch.cuda.synchronize()
-        got = y.double().cpu().numpy().reshape(w.channels, L)
-        assert np.isfinite(got).all(), call
-        err = rel_l2_rows(got, ref)
-        assert err.max() <= TOL[dtype], (call, err.max())
+        assert torch.cuda.mem_get_info()[0] == free_before, call
+        assert torch.cuda.memory_reserved() == reserved_before, call
+        got_bits = y.view(torch.int16 if dtype == "bf16" else torch.int32).cpu().numpy()
+        np.testing.assert_array_equal(got_bits, ref_bits, err_msg=f"call {call}")
+    hy.check_device_timeouts()
+    # one row against the float64 oracle (the last row: the last, partial wave)
+    row = w.channels - 1
+    got = ys[1].float().cpu().numpy().reshape(w.channels, L)[[row]]
+    ref = oracle_rows(w, [row], v, xs, wt)
+    err = rel_l2_rows(got, ref)
+    assert err.max() <= TOL[dtype], err.max()
 
 
 def test_static_workspace_rejects_short_lengths():
@@ -65,3 +87,9 @@ def test_static_workspace_rejects_short_lengths():
         == hy.HYENA_ERR_UNSUPPORTED
     assert lib.hyena_forward_static_workspace(p, arr, arr, 1, 1, 3000, 2, hy.HYENA_F32, p, None) \
         == hy.HYENA_ERR_UNSUPPORTED
+    # misaligned or null pointers are refused on the host, before any lookup
+    mis = ctypes.c_void_p(t.data_ptr() + 4)
+    assert lib.hyena_forward_static_workspace(mis, arr, arr, 1, 1, 32768, 2, hy.HYENA_F32, p, None) \
+        == hy.HYENA_ERR_INVALID_ARG
+    assert lib.hyena_forward_static_workspace(p, None, arr, 1, 1, 32768, 2, hy.HYENA_F32, p, None) \
+        == hy.HYENA_ERR_INVALID_ARG
