@@ -74,7 +74,7 @@ L2_BYTES = 126 * 2 ** 20
 KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
-    "tc": ("tc_fused.cu", "fft_engine.cuh", "layout.h"),
+    "tc": ("tc_fused.cu", "tc_dft.cuh", "fft_engine.cuh", "layout.h"),
 }
 
 

@@ -107,6 +107,14 @@ SWEEP = [
     (2, "bf16", 6, 3, 2048),
     # odd B at a tensor-core length falls back to the SIMT kernel
     (2, "bf16", 3, 2, 2048),
+    # tensor-core four-step: bf16, 2^16 <= L <= 2^20 (rows of R * 256 points, R = 1 .. 16)
+    (1, "bf16", 1, 2, 65536),
+    (2, "bf16", 2, 3, 131072),
+    (3, "bf16", 1, 2, 262144),
+    (3, "bf16", 3, 1, 524288),
+    (2, "bf16", 1, 2, 1048576),
+    # order 4 keeps the float32 four-step kernels at these lengths
+    (4, "bf16", 3, 1, 524288),
 ]
 
 
@@ -120,7 +128,7 @@ def test_forward_shapes(hy, N, dtype, B, D, L):
     assert err.max() <= TOL[dtype], err.max()
 
 
-@pytest.mark.parametrize("L,dtype", [(2048, "f32"), (2048, "bf16"), (32768, "f32")])
+@pytest.mark.parametrize("L,dtype", [(2048, "f32"), (2048, "bf16"), (32768, "f32"), (131072, "bf16")])
 def test_forward_in_place_and_waves(hy, L, dtype):
     import torch
     w = synth.custom(2, dtype, 2, 3, L, seed=5)
@@ -144,7 +152,7 @@ def test_forward_in_place_and_waves(hy, L, dtype):
         txs = [upload(x, w) for x in xs]
         ws = torch.empty(8 * L, dtype=torch.uint8, device="cuda")
         y1 = hy.forward(tv, txs, hh, workspace=ws)
-        np.testing.assert_array_equal(y1.cpu().numpy().reshape(w.channels, L), y_ref)
+        np.testing.assert_array_equal(y1.float().cpu().numpy().reshape(w.channels, L), y_ref)
 
 
 @pytest.mark.parametrize("cfg_i", [1, 2, 3, 4])
