@@ -293,7 +293,7 @@ def forward_f16_spectra(v, xs, hhats16, y=None, workspace=None, stream=None):
 
 
 def forward_static_workspace(v, xs, hhats, y=None, stream=None):
-    """hyena_forward_static_workspace: the long-sequence forward (8192 < L)
+    """hyena_forward_static_workspace: the long-sequence forward (16384 < L)
     with the library's static device scratch instead of a caller workspace,
     for callers that cannot allocate device memory. Calls whose GPU work
     overlaps race on that scratch; the first call on a device must come

@@ -25,14 +25,18 @@ struct FusedOcc {
 };
 
 // Shared memory: z (padded), staged filter spectrum row (bins of type HT),
-// staged gate row, staged v row of the next channel.
+// staged gate row, staged v row of the next channel. At the longest fused
+// length (2^14 points) z alone takes 136 KB, so the spectrum is read from
+// global memory instead of being staged, and for float32 rows v is too.
 template <int LOGMV, typename T, typename HT = float2>
 struct FusedSmem {
   static constexpr int MV = 1 << LOGMV;
+  static constexpr bool stage_h = LOGMV <= 13;
+  static constexpr bool stage_v = LOGMV <= 13 || sizeof(T) < 4;
   static constexpr size_t z = sizeof(float2) * padded_len(MV);
-  static constexpr size_t h = sizeof(HT) * MV;
+  static constexpr size_t h = stage_h ? sizeof(HT) * MV : 0;
   static constexpr size_t row = sizeof(T) * MV;      // L <= MV elements, 16-byte multiple
-  static constexpr size_t total = z + h + 2 * row;
+  static constexpr size_t total = z + h + (stage_v ? 2 : 1) * row;
 };
 
 // Per-channel factor of a spectrum block: 1 for float32 bins; for __half2
@@ -56,7 +60,7 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
   extern __shared__ __align__(16) float2 sm[];
   HT* hs = reinterpret_cast<HT*>(reinterpret_cast<char*>(sm) + S::z);
   T* xs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h);
-  T* vs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h + S::row);
+  T* vs = reinterpret_cast<T*>(reinterpret_cast<char*>(sm) + S::z + S::h + S::row);   // if S::stage_v
   const int tl = threadIdx.x;
   const float2* __restrict__ tw = tables;
   const float2* __restrict__ Wv = tables + MV;
@@ -73,8 +77,8 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
   long long ch = blockIdx.x;
   if (ch < C) {
     const int c = (int)(ch / B), b = (int)(ch % B);
-    block_copy_async(vs, v + ((size_t)b * D + c) * (size_t)L, row_bytes, tl, TV);
-    block_copy_async(hs, spec_row(0, c), h_bytes, tl, TV);
+    if constexpr (S::stage_v) block_copy_async(vs, v + ((size_t)b * D + c) * (size_t)L, row_bytes, tl, TV);
+    if constexpr (S::stage_h) block_copy_async(hs, spec_row(0, c), h_bytes, tl, TV);
     cp_async_commit();
     cp_async_wait_all();
   }
@@ -87,7 +91,10 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int m = tl + r * Q16;
-      a[r] = (2 * m < L) ? IO<T>::load2_smem(vs + 2 * m) : make_float2(0.f, 0.f);
+      if constexpr (S::stage_v)
+        a[r] = (2 * m < L) ? IO<T>::load2_smem(vs + 2 * m) : make_float2(0.f, 0.f);
+      else
+        a[r] = (2 * m < L) ? IO<T>::load2(v + row + 2 * m) : make_float2(0.f, 0.f);
     }
     for (int n = 0; n < N; ++n) {
       // forward: first pass (radix 16, upper half of the input is zero)
@@ -96,7 +103,7 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
       __syncthreads();
       // every thread is past its reads of the gate and v buffers: refill them
       block_copy_async(xs, pick(x, n) + row, row_bytes, tl, TV);
-      if (n == 0 && ch + gridDim.x < C) {
+      if (S::stage_v && n == 0 && ch + gridDim.x < C) {
         const long long nx = ch + gridDim.x;
         const int c2 = (int)(nx / B), b2 = (int)(nx % B);
         block_copy_async(vs, v + ((size_t)b2 * D + c2) * (size_t)L, row_bytes, tl, TV);
@@ -107,10 +114,15 @@ fused_forward_kernel(const T* __restrict__ v, GatePtrs<T> x, SpecPtrs hh, T* __r
       cp_async_wait_all();
       __syncthreads();
       // last forward pass + spectral product + first inverse pass
-      paired_pass<LOGMV, kPairConv, true, HT>(sm, sm, jA, jB, head, tw, Wv, one, false, hs, hs, 0.f);
+      if constexpr (S::stage_h) {
+        paired_pass<LOGMV, kPairConv, true, HT>(sm, sm, jA, jB, head, tw, Wv, one, false, hs, hs, 0.f);
+      } else {
+        HT* hg = const_cast<HT*>(spec_row(n, c));
+        paired_pass<LOGMV, kPairConv, false, HT>(sm, sm, jA, jB, head, tw, Wv, one, false, hg, hg, 0.f);
+      }
       __syncthreads();
       // the spectrum buffer is free: stage the next spectrum (next stage or next channel)
-      {
+      if constexpr (S::stage_h) {
         const HT* hn = nullptr;
         if (n + 1 < N) {
           hn = spec_row(n + 1, c);
@@ -211,6 +223,7 @@ cudaError_t launch_fused_forward(const FusedLaunch& p, int logMV, cudaStream_t s
     case 11: return launch_fused_l<11>(p, s);
     case 12: return launch_fused_l<12>(p, s);
     case 13: return launch_fused_l<13>(p, s);
+    case 14: return launch_fused_l<14>(p, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -239,6 +252,7 @@ cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* ta
     case 11: return launch_fused_spec_l<11>(h, spec, tables, D, L, s);
     case 12: return launch_fused_spec_l<12>(h, spec, tables, D, L, s);
     case 13: return launch_fused_spec_l<13>(h, spec, tables, D, L, s);
+    case 14: return launch_fused_spec_l<14>(h, spec, tables, D, L, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -9,7 +9,7 @@ namespace hyena {
 
 // Lengths up to this run the fused per-channel kernel (whole channel in shared
 // memory); longer ones run the four-step decomposition through a workspace.
-constexpr int kFusedMaxL = 8192;
+constexpr int kFusedMaxL = 16384;
 constexpr int kMinM = 128;          // smallest internal transform (zero-extended below)
 constexpr int kMaxL = 1 << 20;
 constexpr int kFourStepMaxMV = 4096;

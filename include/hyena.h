@@ -118,10 +118,11 @@ hyena_status hyena_filter_rfft(const float *h, int D, int L, void *hhat, hyena_s
 hyena_status hyena_spectrum_layout(int L, int *M, int *M1, int *MV);
 
 /*
- * Workspace bytes hyena_forward wants for this shape: 0 for L <= 8192 (the
+ * Workspace bytes hyena_forward wants for this shape: 0 for L <= 16384 (the
  * fused kernel keeps everything on chip); for longer L, 8*L bytes per
- * channel for a wave of channels sized to stay resident in L2. Any workspace
- * of at least 8*L bytes works (smaller waves); 0 when the shape is invalid.
+ * channel for a wave of channels sized to stay resident in L2 (3/4 of the
+ * current device's L2 capacity). Any workspace of at least 8*L bytes works
+ * (smaller waves); 0 when the shape is invalid.
  */
 size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dtype);
 
@@ -133,7 +134,7 @@ size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dty
  *         hyena_filter_rfft (D channels, the same L)
  *   y:    device [B][D][L] dtype; may alias v or any x[n] (each element is
  *         read before the same thread block writes it)
- *   workspace: device scratch of workspace_bytes (>= 8*L when L > 8192;
+ *   workspace: device scratch of workspace_bytes (>= 8*L when L > 16384;
  *         ignored otherwise, may be NULL)
  */
 hyena_status hyena_forward(const void *v, const void *const *x, const void *const *hhat, int B, int D, int L,
@@ -158,7 +159,7 @@ hyena_status hyena_forward(const void *v, const void *const *x, const void *cons
  * phase that must not reserve memory) -- and held until the process exits.
  * A call rejected by the host-side checks loads nothing.
  *
- *  - Only for 8192 < L <= 2^20 (the lengths whose forward needs scratch);
+ *  - Only for 16384 < L <= 2^20 (the lengths whose forward needs scratch);
  *    shorter L returns HYENA_ERR_UNSUPPORTED: use hyena_forward with a NULL
  *    workspace there, which already allocates nothing.
  *  - Channels are processed in waves of HYENA_STATIC_WORKSPACE_BYTES / (8 L);

@@ -80,7 +80,8 @@ SWEEP = [
     (2, "bf16", 2, 3, 1024),
     (2, "f32", 3, 2, 2048),
     (3, "bf16", 2, 2, 8192),
-    (2, "f32", 1, 2, 16384),     # four-step
+    (2, "f32", 1, 2, 16384),     # fused, 1024 threads per channel
+    (2, "f32", 1, 2, 32768),     # four-step
     (2, "bf16", 2, 1, 32768),    # four-step
 ]
 

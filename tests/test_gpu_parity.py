@@ -64,12 +64,12 @@ def test_spectrum_matches_oracle(hy, L):
 @pytest.mark.parametrize("cfg_i,nsample", [(0, None), (1, 24), (2, 12), (3, None), (4, None)])
 def test_forward_workload(hy, cfg_i, nsample):
     """Full-size workloads in the bench's launch configuration. The four-step
-    workloads (L > 8192) are checked on one seeded row of every wave of
+    workloads (L > 16384) are checked on one seeded row of every wave of
     channels the default workspace holds, plus the first and last rows."""
     w = synth.workload(cfg_i)
     y, _, (v, xs, wt) = gpu_run(w)
     assert np.isfinite(y).all()
-    if w.L > 8192:
+    if w.L > 16384:
         ws = hy.forward_workspace_bytes(w.B, w.D, w.L, w.N, w.dtype == "bf16")
         wave = ws // (8 * w.L)
         assert wave >= 1
@@ -94,7 +94,11 @@ SWEEP = [
     (3, "f32", 2, 2, 1024),
     (1, "f32", 2, 2, 4096),
     (2, "f32", 1, 3, 8192),
+    # the fused on-chip kernel at its longest length (1024 threads per channel)
     (2, "f32", 1, 2, 16384),
+    (3, "f32", 3, 2, 16384),
+    (2, "bf16", 1, 3, 16384),
+    (2, "bf16", 3, 2, 16384),
     (3, "bf16", 1, 3, 32768),
     (2, "f32", 2, 1, 65536),
     (1, "f32", 1, 2, 262144),
@@ -146,7 +150,7 @@ def test_forward_in_place_and_waves(hy, L, dtype):
     tv = upload(v, w)
     hy.forward(tv, txs, hh, y=txs[-1])
     np.testing.assert_array_equal(txs[-1].float().cpu().numpy().reshape(w.channels, L), y_ref)
-    if L > 8192:
+    if L > 16384:
         # a one-channel workspace: every channel runs in its own wave
         tv = upload(v, w)
         txs = [upload(x, w) for x in xs]
@@ -192,3 +196,34 @@ def test_forward_is_deterministic_and_scales_exactly(hy, cfg_i):
     y4 = hy.forward(tv * 4, txs, hh)
     assert torch.equal(y1, y2)
     assert torch.equal(y4, y1 * 4)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fused_dispatch_up_to_16384(hy, dtype):
+    """L = 16384 runs the fused on-chip kernel: no workspace is asked for and
+    one forward is one kernel launch (counted from a CUDA-graph capture)."""
+    import torch
+    import cuda.bindings.runtime as rt
+    assert hy.forward_workspace_bytes(2, 3, 16384, 2, dtype == "bf16") == 0
+    assert hy.forward_workspace_bytes(2, 3, 32768, 2, dtype == "bf16") > 0
+    w = synth.custom(2, dtype, 2, 3, 16384, seed=9)
+    wt = synth.filter_weights(w)
+    v, xs = synth.inputs(w)
+    h = hy.filter_generate(weights_to_cuda(wt), w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
+    hh = [hy.filter_rfft(h[n]) for n in range(w.N)]
+    tv = upload(v, w)
+    txs = [upload(x, w) for x in xs]
+    y = torch.empty_like(tv)
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        hy.forward(tv, txs, hh, y=y, stream=side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        hy.forward(tv, txs, hh, y=y, stream=side)
+    graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+    _, _, n = rt.cudaGraphGetNodes(graph, 0)
+    _, nodes, n = rt.cudaGraphGetNodes(graph, n)
+    kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    assert sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel) == 1
+    g.reset()

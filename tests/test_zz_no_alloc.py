@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("N,dtype,B,D,L", [(2, "bf16", 2, 3, 32768), (2, "bf16", 1, 40, 131072),
-                                           (3, "f32", 1, 2, 16384), (2, "bf16", 1, 3, 1 << 20)])
+                                           (3, "f32", 1, 2, 32768), (2, "bf16", 1, 3, 1 << 20)])
 def test_static_workspace_matches_workspace_forward(N, dtype, B, D, L):
     import torch
     from fft_long_convolution_implicit_b200 import build
@@ -84,6 +84,8 @@ def test_static_workspace_rejects_short_lengths():
     p = ctypes.c_void_p(t.data_ptr())
     arr = (ctypes.c_void_p * 2)(t.data_ptr(), t.data_ptr())
     assert lib.hyena_forward_static_workspace(p, arr, arr, 1, 1, 2048, 2, hy.HYENA_F32, p, None) \
+        == hy.HYENA_ERR_UNSUPPORTED
+    assert lib.hyena_forward_static_workspace(p, arr, arr, 1, 1, 16384, 2, hy.HYENA_F32, p, None) \
         == hy.HYENA_ERR_UNSUPPORTED
     assert lib.hyena_forward_static_workspace(p, arr, arr, 1, 1, 3000, 2, hy.HYENA_F32, p, None) \
         == hy.HYENA_ERR_UNSUPPORTED
