@@ -17,15 +17,17 @@ namespace hyena {
 
 enum PairMode { kPairConv = 0, kPairSpectrum = 1 };
 
-// Filter spectrum reads: from global memory through the read-only path, or
-// from a shared-memory copy staged by the caller (H_SMEM); bins stored as
-// float2, or as __half2 (the reduced-precision block, scaled per channel by
-// a power of two that the caller removes at the gate).
+// Filter spectrum reads: from global memory as streaming loads (each bin is
+// read once per forward, so it is marked evict-first and does not displace
+// the four-step scratch from L2), or from a shared-memory copy staged by the
+// caller (H_SMEM); bins stored as float2, or as __half2 (the reduced-precision
+// block, scaled per channel by a power of two that the caller removes at the
+// gate).
 template <bool H_SMEM, typename HT = float2>
 struct HRead;
 template <>
 struct HRead<false, float2> {
-  static __device__ __forceinline__ float2 at(const float2* p, int i) { return __ldg(p + i); }
+  static __device__ __forceinline__ float2 at(const float2* p, int i) { return __ldcs(p + i); }
 };
 template <>
 struct HRead<true, float2> {
@@ -33,7 +35,7 @@ struct HRead<true, float2> {
 };
 template <>
 struct HRead<false, __half2> {
-  static __device__ __forceinline__ float2 at(const __half2* p, int i) { return __half22float2(__ldg(p + i)); }
+  static __device__ __forceinline__ float2 at(const __half2* p, int i) { return __half22float2(__ldcs(p + i)); }
 };
 template <>
 struct HRead<true, __half2> {
