@@ -80,7 +80,7 @@ KERNEL_FILES = {
 
 def dominant_kernel(w: synth.Workload, spec16: bool = False) -> tuple[str, str]:
     """(kernel name, source set) of the launch that dominates one forward."""
-    if w.L > 8192:
+    if w.L > 16384:
         return "four-step column/row kernels (whole step)", "fourstep"
     if spec16:
         return "fused_forward_kernel (f16 spectra)", "fused"
