@@ -24,8 +24,20 @@
 namespace hyena {
 
 // ------------------------------------------------------------------ complex --
+// Complex sums and differences as one packed f32x2 instruction each (exactly
+// rounded per component, the same values as two scalar operations; the
+// difference is a - b = fma(b, -1, a), exact too), which halves the issue
+// slots of the butterflies' additions.
+#ifndef HYENA_PACKED_ADD
+#define HYENA_PACKED_ADD 1
+#endif
+#if HYENA_PACKED_ADD
+__device__ __forceinline__ float2 cadd(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 csub(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
+#else
 __device__ __forceinline__ float2 cadd(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
 __device__ __forceinline__ float2 csub(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
+#endif
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
   return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
