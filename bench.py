@@ -214,6 +214,29 @@ def rank_workload(w: synth.Workload, rank: int) -> synth.Workload:
     return synth.Workload(**{**w.__dict__, "seed": w.seed + 7919 * rank})
 
 
+def default_steps(torch, step, stream, target_s: float = 20.0) -> int:
+    """Timed steps when --steps is not given: enough for about target_s
+    seconds of timed work, from the mean of three untimed steps (at least 20,
+    at most 20000). Under several ranks the smallest count is taken (a MIN
+    all-reduce before the timed region), so that every rank times the same
+    number of steps."""
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(3):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    per = max(a.elapsed_time(b) / 3.0, 1e-3) * 1e-3
+    k = int(min(20000, max(20, target_s / per)))
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        t = torch.tensor([k], device=torch.device("cuda", torch.cuda.current_device()), dtype=torch.int64)
+        dist.all_reduce(t, op=dist.ReduceOp.MIN)
+        k = int(t.item())
+    return k
+
+
 def max_over_ranks(value: float, dist, device) -> float:
     """Max of a per-rank float over all ranks (identity without a process group)."""
     if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
@@ -425,6 +448,8 @@ def run_nd(args) -> int:
     if args.impl == "reference":
         if rank != 0:
             return 0
+        if args.steps is None:
+            args.steps = 20
         import oracle
         K = synth.nd_kernels(w)
 
@@ -503,6 +528,8 @@ def run_nd(args) -> int:
     for i in range(args.warmup):
         sets[i % nsets]()
     torch.cuda.synchronize()
+    if args.steps is None:
+        args.steps = default_steps(torch, lambda i: sets[i % nsets](), stream)
     sampler = ClockSampler(local_rank if world > 1 else 0)
     sampler.start()
     time.sleep(0.2)
@@ -651,8 +678,9 @@ def filter_gen_flops(w: synth.Workload) -> int:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for about 20 s of timed work, 20 to 20000)")
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4,
                     help="workload index (default 4: the largest one-GPU workload, B=1 D=256 L=2^20 N=2 bf16)")
@@ -686,6 +714,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     spec16 = args.spectrum == "f16" and args.which == "forward"
+    if args.impl == "reference" and args.steps is None:
+        args.steps = 20
     if args.impl == "reference":
         if rank != 0:
             return 0
@@ -777,6 +807,8 @@ def main():
     for i in range(args.warmup):
         sets[i % nsets]()
     torch.cuda.synchronize()
+    if args.steps is None:
+        args.steps = default_steps(torch, lambda i: sets[i % nsets](), stream)
 
     sampler = ClockSampler(local_rank if world > 1 else 0)
     sampler.start()
