@@ -75,6 +75,7 @@ KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "fourstep": ("fourstep.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
     "tc": ("tc_fused.cu", "tc_dft.cuh", "fft_engine.cuh", "layout.h"),
+    "tcg": ("tc_gemm.cu", "fft_engine.cuh", "layout.h"),
 }
 
 
@@ -86,6 +87,8 @@ def dominant_kernel(w: synth.Workload, spec16: bool = False) -> tuple[str, str]:
         return "fused_forward_kernel (f16 spectra)", "fused"
     if w.dtype == "bf16" and w.B % 2 == 0 and 1024 <= w.L <= 2048:
         return "tc_forward_kernel", "tc"
+    if w.dtype == "bf16" and w.B % 2 == 0 and w.L == 8192:
+        return "tcg_forward_kernel", "tcg"
     return "fused_forward_kernel", "fused"
 
 

@@ -98,11 +98,11 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     p.B = B; p.D = D; p.L = ly.L; p.N = N;
     p.bf16 = bf16;
     p.spec16 = spec16;
-    if (allow_tc && ly.tc && p.bf16 && (B % 2) == 0) {
+    if (allow_tc && has_tc_copy(ly) && p.bf16 && (B % 2) == 0) {
       // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
       for (int n = 0; n < N; ++n)
         p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);
-      e = launch_tc_forward(p, ly, s);
+      e = ly.tcg ? launch_tcg_forward(p, s) : launch_tc_forward(p, ly, s);
     } else {
       e = launch_fused_forward(p, ly.logMV, s);
     }
@@ -168,6 +168,8 @@ cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, con
     e = launch_fused_spectrum(h, spec, tables, rows, ly.L, ly.logMV, s);
     if (e == cudaSuccess && with_tc && ly.tc)
       e = launch_tc_spectrum(spec, spec + tc_spectrum_offset(ly, rows), tables, rows, ly, s);
+    if (e == cudaSuccess && with_tc && ly.tcg)
+      e = launch_tcg_spectrum(spec, spec + tc_spectrum_offset(ly, rows), rows, s);
   } else {
     for (long long c0 = 0; c0 < rows && e == cudaSuccess; c0 += kMaxGridY) {
       const int nd = (int)((rows - c0) < kMaxGridY ? (rows - c0) : kMaxGridY);
@@ -198,7 +200,9 @@ const char* hyena_last_cuda_error(void) { return g_last_cuda_error; }
 hyena_status hyena_device_timeouts(void) {
   const int b = striped_read_and_clear_timeout();
   if (b < 0) return cuda_fail(cudaGetLastError());
-  return b ? HYENA_ERR_TIMEOUT : HYENA_OK;
+  const int g = tcg_read_and_clear_timeout();
+  if (g < 0) return cuda_fail(cudaGetLastError());
+  return (b || g) ? HYENA_ERR_TIMEOUT : HYENA_OK;
 }
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {

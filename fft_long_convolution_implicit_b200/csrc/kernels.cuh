@@ -86,6 +86,10 @@ cudaError_t launch_fused_spectrum(const float* h, float2* spec, const float2* ta
 cudaError_t launch_tc_forward(const FusedLaunch& p, const Layout& y, cudaStream_t s);
 cudaError_t launch_tc_spectrum(const float2* nat, float2* tcs, float2* tables, int D, const Layout& y,
                                cudaStream_t s);
+// tcgen05 GEMM-level kernel (bf16, L = kTcgL, B even) and its spectrum copy
+cudaError_t launch_tcg_forward(const FusedLaunch& p, cudaStream_t s);
+cudaError_t launch_tcg_spectrum(const float2* nat, float2* tcs, int D, cudaStream_t s);
+int tcg_read_and_clear_timeout();
 // StripedHyena-form operator: featurizer length <= kMaxStripedLF, explicit
 // inner filter length <= kMaxStripedLG. hG == nullptr: featurize only (q, u).
 constexpr int kMaxStripedLF = 16;

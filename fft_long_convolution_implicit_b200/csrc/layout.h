@@ -29,8 +29,10 @@ struct Layout {
   int tw_v;     // MV-point plan twiddles (MV entries)
   int w_v;      // w_{2 MV}^k, k < MV
   int tw_1;     // M1-point column plan twiddles (M1 entries, four-step only)
-  // tensor-core path (bf16, pairs of batch items): 2L = R0 * 256
+  // tensor-core paths (bf16, pairs of batch items): mma.sync kernel with
+  // 2L = R0 * 256 (tc), or tcgen05 GEMM levels 2L = 16 * 32 * 32 (tcg)
   bool tc;
+  bool tcg;
   int R0;
   int tc_otw;   // outer twiddles w_{2L}^{m k0}, [k0 = 1..R0-1][m < 256] (R0 * 256 entries)
   int table_len;
@@ -39,6 +41,8 @@ struct Layout {
 // Lengths with a tensor-core forward (outer radix R0 = L / 128 in {8, 16}).
 constexpr int kTcMinL = 1024;
 constexpr int kTcMaxL = 2048;
+// Length of the tcgen05 GEMM-level forward.
+constexpr int kTcgL = 8192;
 
 inline int ilog2_exact(int v) {
   int l = 0;
@@ -75,6 +79,7 @@ inline bool make_layout(int L, Layout* out) {
   y.tw_1 = 2 * y.MV;
   y.table_len = 2 * y.MV + (y.fourstep ? y.M1 : 0);
   y.tc = (L >= kTcMinL && L <= kTcMaxL);
+  y.tcg = (L == kTcgL);
   y.R0 = y.tc ? L / 128 : 0;
   y.tc_otw = y.table_len;
   if (y.tc) y.table_len += y.R0 * 256;
@@ -84,13 +89,15 @@ inline bool make_layout(int L, Layout* out) {
 }
 
 // One filter's spectrum block: [D][M] float2 spectrum (library order); for
-// tensor-core lengths a second copy [D][L] in the tensor-core order; then the
-// table region.
-// tensor-core copy: rows of L + 2 float2 (L bins, then (1/f_c, 0) and padding)
+// tensor-core lengths a second copy [D][L + 2] float2 in the kernel's order;
+// then the table region.
+// tensor-core copy rows: L float2 bins (mma.sync kernel) or 2L f16x2 bins
+// (tcgen05 kernel), then the channel's 1 / f_c and padding (16 bytes)
 inline int tc_row(const Layout& y) { return y.L + 2; }
+inline bool has_tc_copy(const Layout& y) { return y.tc || y.tcg; }
 inline size_t tc_spectrum_offset(const Layout& y, int D) { return (size_t)D * y.M; }
 inline size_t tables_offset(const Layout& y, int D) {
-  return (size_t)D * y.M + (y.tc ? (size_t)D * tc_row(y) : 0);
+  return (size_t)D * y.M + (has_tc_copy(y) ? (size_t)D * tc_row(y) : 0);
 }
 inline size_t spectrum_block_floats2(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
 

@@ -1,0 +1,642 @@
+// tc_gemm.cu -- Hyena order-N forward for bf16 I/O at L = 8192, B even, with
+// every DFT level of the transform as a GEMM on the 5th-generation tensor
+// cores (tcgen05.mma: f16 operands in shared memory, f32 accumulators in TMEM).
+//
+// Two batch items b, b+1 of channel c share the filter h_c, so their causal
+// convolutions are the real and imaginary parts of one complex convolution of
+// c[m] = z_b[m] + i z_{b+1}[m] on the 2L zero-padded grid (glossary
+// "Hyena（ハイエナ）", section 計算効率; "Native Multi-Dimensional Subquadratic
+// Operators via Input Dependent Long Convolutions", section 境界の処理).
+// With P = 2L = 16384 = 16 * 32 * 32, m = m'' + 32 n2 + 1024 n3 and
+// k = k3 + 16 k2 + 512 k1 (a Cooley-Tukey split written as three levels):
+//   F1  rows m' = m'' + 32 n2 (1024): 16-point DFT over n3 (n3 < 8 nonzero),
+//       then the twiddle w_P^{m' k3};
+//   F2  rows (k3, m'') (512): 32-point DFT over n2, twiddle w_1024^{m'' k2};
+//   F3  rows (k3, k2) (512): 32-point DFT over m'' -> C[k];
+//   the product with the filter spectrum (an f16 copy in F3-row order);
+//   I3  rows (k3, k2): inverse 32-point DFT over k1 -> m'', twiddle w_1024^{-m'' k2};
+//   I2  rows (k3, m''): inverse 32-point DFT over k2 -> n2, twiddle w_P^{-m' k3};
+//   I1  rows m': inverse 16-point DFT over k3, outputs n3 < 8 only (t < L).
+// Each level is D[rows x 2R] = A[rows x 2K] B[2R x 2K]^T with complex values
+// interleaved (re, im) along K and N, so the real form of the DFT matrix in B
+// carries the complex arithmetic. A thread owns fixed TMEM rows in every level
+// (warp w reads lanes 32 (w % 4) .. + 31 of the tiles of parity w / 4): it
+// reads its rows of D (tcgen05.ld), applies the twiddles in fp32 (powers by
+// recurrence from per-thread bases) and writes the values into the rows of the
+// next level's A operand; the row numberings and the operand strides are chosen
+// so that every one of these stores is free of shared-memory bank conflicts.
+// The output rows of I1 are the input rows of F1, so z stays in registers
+// between the N stages. One thread issues the MMAs; completion arrives on an
+// mbarrier through tcgen05.commit; every wait is bounded in time.
+//
+// Scaling (exact powers of two): z is scaled so max |component| < 2^6, which
+// keeps every f16 operand of F1..F3 below 2^15; the spectrum copy is scaled per
+// channel to [2^14, 2^15) and the product by 2^-30, which keeps I3..I1 below
+// 2^15; all factors are removed at the gate.
+#include <cuda_fp16.h>
+
+#include "fft_engine.cuh"
+#include "kernels.cuh"
+
+namespace hyena {
+
+namespace {
+
+constexpr int kGT = 256;                  // threads per CTA
+constexpr int kGL = 8192;                 // L
+constexpr int kGP = 2 * kGL;              // transform length
+constexpr uint32_t kGCols = 256;          // TMEM columns per CTA
+// A operand (K-major, no swizzle, core matrices of 8 rows x 16 B): byte
+// address of complex element kappa of row r within a 128-row tile is
+//   (r & 7) * 16 + (kappa & 3) * 4 + (kappa >> 2) * LBO + (r >> 3) * SBO.
+constexpr uint32_t kF1Lbo = 128, kF1Sbo = 256, kF1Tile = 16 * 256;        // rows of 8 complex
+constexpr uint32_t kCLbo = 128, kCSbo = 1024, kCTile = 16 * 1024;         // rows of 32 complex (F2, I3, I2)
+constexpr uint32_t kF3Lbo = 2064, kF3Sbo = 128, kF3Tile = 8 * 2064;       // F3: K chunks 2064 B apart
+constexpr uint32_t kI1Lbo = 2080, kI1Sbo = 128, kI1Tile = 4 * 2080;       // I1: K chunks 2080 B apart
+constexpr uint32_t kABytes = 66560;
+static_assert(4 * kF3Tile <= kABytes && 8 * kI1Tile <= kABytes && 4 * kCTile <= kABytes, "A region");
+// B operands (DFT matrices, K-major canonical: LBO 128, SBO = K / 8 * 128)
+constexpr uint32_t kBF1 = 0;              // forward 16-point, inputs < 8: N 32 x K 16
+constexpr uint32_t kBF32 = 1024;          // forward 32-point: N 64 x K 64
+constexpr uint32_t kBI32 = 9216;          // inverse 32-point: N 64 x K 64
+constexpr uint32_t kBI1 = 17408;          // inverse 16-point, outputs < 8: N 16 x K 32
+constexpr uint32_t kBBytes = 18432;
+constexpr uint32_t kOffA = 0;
+constexpr uint32_t kOffB = kABytes;
+constexpr uint32_t kOffMisc = kOffB + kBBytes;   // mbarrier, TMEM address, 8 partial maxima
+constexpr uint32_t kOffPtr = kOffMisc + 64;      // gate and spectrum pointers of the N stages
+constexpr uint32_t kGSmem = kOffPtr + 16 * kMaxOrder;
+// spectrum copy row: 2L f16x2 bins in F3-row order, then 1 / f_c (float), padding
+constexpr size_t kGHRowBytes = (size_t)4 * kGP + 16;
+
+// instruction descriptor: f32 accumulate, f16 A and B, both K-major, M = 128
+__host__ __device__ constexpr uint32_t g_idesc(int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t g_smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t g_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46);
+}
+
+__device__ __forceinline__ void g_mma(uint32_t dtmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(dtmem),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+__device__ __forceinline__ void g_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long g_globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for an mbarrier phase, bounded in time (each try suspends at most
+// 20 us; false once limit_ns of global time have passed).
+constexpr unsigned long long kGWaitLimitNs = 200000000ull;   // 0.2 s
+__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t phase, unsigned long long limit_ns = kGWaitLimitNs) {
+  const unsigned long long t0 = g_globaltimer_ns();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, P1;\n\t}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(phase), "r"(20000u)
+        : "memory");
+    if (done) return true;
+    if (g_globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+#define G_LD_REGS16(r, o)                                                                                      \
+  "=r"(r[o + 0]), "=r"(r[o + 1]), "=r"(r[o + 2]), "=r"(r[o + 3]), "=r"(r[o + 4]), "=r"(r[o + 5]),              \
+      "=r"(r[o + 6]), "=r"(r[o + 7]), "=r"(r[o + 8]), "=r"(r[o + 9]), "=r"(r[o + 10]), "=r"(r[o + 11]),        \
+      "=r"(r[o + 12]), "=r"(r[o + 13]), "=r"(r[o + 14]), "=r"(r[o + 15])
+
+// 32 consecutive TMEM columns of this thread's lane (not yet waited for)
+__device__ __forceinline__ void g_ld32(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : G_LD_REGS16(r, 0), G_LD_REGS16(r, 16)
+      : "r"(addr));
+}
+__device__ __forceinline__ void g_ld16(uint32_t addr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : G_LD_REGS16(r, 0)
+      : "r"(addr));
+}
+__device__ __forceinline__ void g_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+#undef G_LD_REGS16
+
+__device__ __forceinline__ uint32_t g_pack(float re, float im) {
+  const __half2 v = __floats2half2_rn(re, im);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// a * b with packed f32x2 arithmetic: (a.x b.x - a.y b.y, a.x b.y + a.y b.x)
+__device__ __forceinline__ float2 g_cmul(float2 a, float2 b) {
+  const float2 t = __fmul2_rn(make_float2(a.y, a.y), make_float2(-b.y, b.x));
+  return __ffma2_rn(make_float2(a.x, a.x), b, t);
+}
+
+// The twiddle powers of a recurrence depend only on per-thread constants; a
+// compiler that hoists them out of the pair and stage loops holds dozens of
+// them in registers for the whole kernel. Passing the base through an opaque
+// move keeps each recurrence where its powers are used.
+__device__ __forceinline__ float2 g_opaque(float2 a) {
+  float2 b;
+  asm volatile("mov.b32 %0, %2;\n\tmov.b32 %1, %3;" : "=f"(b.x), "=f"(b.y) : "f"(a.x), "f"(a.y));
+  return b;
+}
+
+__device__ __forceinline__ float2 g_cval(const uint32_t (&r)[32], int j) {
+  return make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+}
+
+// w_n^{e} = exp(-2 pi i e / n) for an exact integer e (|e| < n)
+__device__ __forceinline__ float2 g_root(int e, int n) {
+  float s, c;
+  sincospif(-2.0f * (float)e / (float)n, &s, &c);
+  return make_float2(c, s);
+}
+
+// Power of two s with mx * s < 2^6 (>= 2^5 for mx > 0), and 1 / s.
+__device__ __forceinline__ void g_scale_in(float mx, float& s, float& inv_s) {
+  int e = (int)((__float_as_uint(mx) >> 23) & 0xff);   // mx < 2^(e - 126)
+  e = e < 6 ? 6 : (e > 254 ? 254 : e);
+  s = __uint_as_float((unsigned)(259 - e > 254 ? 254 : 259 - e) << 23);   // 2^(132 - e)
+  inv_s = __uint_as_float((unsigned)(e - 5) << 23);                        // 2^(e - 132)
+  if (mx == 0.f) { s = 1.f; inv_s = 1.f; }
+}
+
+__device__ int g_tcg_timeout;
+
+// DFT-matrix operand element (n, k) of a K-major canonical B operand with K f16 columns.
+__device__ __forceinline__ void g_put(unsigned char* sB, uint32_t base, int K, int n, int k, float v) {
+  const uint32_t o = base + (uint32_t)((n & 7) * 16 + (k & 7) * 2 + (k >> 3) * 128 + (n >> 3) * (K / 8) * 128);
+  *reinterpret_cast<__half*>(sB + o) = __float2half_rn(v);
+}
+
+// Real form of F[o][i] = w_n^{sign o i} (outputs o < no, inputs i < ni) at `base`:
+// rows 2o + rho, columns 2i + sigma: [[Fr, -Fi], [Fi, Fr]].
+__device__ void g_build_dft(unsigned char* sB, uint32_t base, int n, int no, int ni, bool inverse, int tid) {
+  const int K = 2 * ni;
+  for (int idx = tid; idx < no * ni; idx += kGT) {
+    const int o = idx / ni, i = idx % ni;
+    const int e = (o * i) % n;
+    float2 w = g_root(e, n);
+    if (inverse) w.y = -w.y;
+    g_put(sB, base, K, 2 * o, 2 * i, w.x);
+    g_put(sB, base, K, 2 * o, 2 * i + 1, -w.y);
+    g_put(sB, base, K, 2 * o + 1, 2 * i, w.y);
+    g_put(sB, base, K, 2 * o + 1, 2 * i + 1, w.x);
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kGT, 2)
+tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> x, SpecPtrs hh,
+                   __nv_bfloat16* __restrict__ y, int B, int D, int N, long long npairs) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, q = w & 3, hw = w >> 2;
+  unsigned char* sA = sm + kOffA;
+  unsigned char* sB = sm + kOffB;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kOffMisc);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kOffMisc + 8);
+  float* red = reinterpret_cast<float*>(sm + kOffMisc + 16);
+  const __nv_bfloat16** xptr = reinterpret_cast<const __nv_bfloat16**>(sm + kOffPtr);
+  const unsigned char** hptr = reinterpret_cast<const unsigned char**>(sm + kOffPtr + 8 * kMaxOrder);
+  const uint32_t aA = g_smem_u32(sA), aB = g_smem_u32(sB), abar = g_smem_u32(bar);
+
+  if (w == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(g_smem_u32(tslot)),
+                 "r"(kGCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+  }
+  if (tid < kMaxOrder) {
+    xptr[tid] = x.p[tid];
+    hptr[tid] = reinterpret_cast<const unsigned char*>(hh.p[tid]);
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(abar), "r"(1));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  g_build_dft(sB, kBF1, 16, 16, 8, false, tid);
+  g_build_dft(sB, kBF32, 32, 32, 32, false, tid);
+  g_build_dft(sB, kBI32, 32, 32, 32, true, tid);
+  g_build_dft(sB, kBI1, 16, 8, 16, true, tid);
+
+  // ---- per-thread row ownership, twiddle bases and store addresses
+  // F1 / I1 rows i: m' = l + 128 w + 32 i (tile 2i + hw); time t = m' + 1024 n3
+  // (rows i > 0: tw1 * w_512^i)
+  const float2 tw1 = g_root(l + 128 * w, kGP);
+  // F2 rows t: (k3 = q + 4 hw + 8 t, m'' = l); twiddle base w_1024^{l}
+  const float2 tw2 = g_root(l, 1024);
+  // F3 / I3 rows t: (k3 = 8 hw + (l >> 2), k2 = (l & 3) + 4 q + 16 t); I3 twiddle base w_1024^{-k2}
+  const float2 tw3a = g_root(-((l & 3) + 4 * q), 1024), tw3b = g_root(-((l & 3) + 4 * q + 16), 1024);
+  // I2 rows t: (k3 = l & 15, m'' = (l >> 4) + 2 q + 8 hw + 16 t);
+  // twiddle w_P^{-(m'' + 32 n2) k3} = start_t * base^{n2}
+  const int k3i2 = l & 15;
+  const float2 st2a = g_root(-(((l >> 4) + 2 * q + 8 * hw) * k3i2), kGP);
+  const float2 st2b = g_root(-(((l >> 4) + 2 * q + 8 * hw + 16) * k3i2), kGP);
+  const float2 tw2i = g_root(-32 * k3i2, kGP);
+
+  // byte offsets (A region) of this thread's stores
+  const uint32_t f1_base = (uint32_t)((l & 7) * 16 + (16 * hw + 4 * q + (l >> 3)) * kF1Sbo);   // + c*128 + i*8192
+  const uint32_t f12_base = (uint32_t)((l & 7) * 16 + w * 128 + (l >> 3) * 1024);           // + 4096 k3
+  // row t of each level adds t times the second constant
+  const uint32_t f23_base = (uint32_t)(64 * (q & 1) + 128 * ((q >> 1) + 2 * hw) + (l & 3) * 4 + (l >> 2) * kF3Lbo);
+  constexpr uint32_t f23_step = kF3Tile;
+  const uint32_t i3_base = (uint32_t)((l & 7) * 16 + (16 * hw + 4 * q + (l >> 3)) * kCSbo);   // + c*128
+  constexpr uint32_t i3_step = 32 * kCSbo;
+  const uint32_t i32_base = (uint32_t)((l >> 2) * 16 + (l & 3) * 4 + q * 128 + hw * 1024);
+  constexpr uint32_t i32_step = 4 * 128;
+  const uint32_t i21_base = (uint32_t)((((l >> 4) + 2 * q) * 16) + (k3i2 & 3) * 4 + (k3i2 >> 2) * kI1Lbo + hw * 128);
+  constexpr uint32_t i21_step = 2 * 128;
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+  const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16);
+
+  uint32_t phase = 0;
+  bool ok = true;       // this thread's last wait completed
+  // One MMA level: every thread's operand stores are made visible to the
+  // tensor core, thread 0 issues `issue`, all wait for completion.
+  auto level = [&](auto issue) -> bool {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    const int bad = __syncthreads_or(ok ? 0 : 1);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (bad) return false;
+    if (tid == 0) {
+      issue();
+      g_commit(abar);
+    }
+    ok = g_wait(abar, phase);
+    phase ^= 1;
+    if (!ok) atomicExch(&g_tcg_timeout, 1);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    return true;
+  };
+  auto issue_f1 = [&]() {
+#pragma unroll 1
+    for (int T = 0; T < 8; ++T)
+      g_mma(tmem + 32u * T, g_desc(aA + T * kF1Tile, kF1Lbo, kF1Sbo), g_desc(aB + kBF1, 128, 256), g_idesc(32), 0u);
+  };
+  auto issue_c = [&](uint32_t tile, uint32_t lbo, uint32_t sbo, uint32_t bmat) {
+#pragma unroll 1
+    for (int T = 0; T < 4; ++T)
+#pragma unroll 1
+      for (int s = 0; s < 4; ++s)
+        g_mma(tmem + 64u * T, g_desc(aA + T * tile + s * 2 * lbo, lbo, sbo), g_desc(aB + bmat + s * 256, 128, 1024),
+              g_idesc(64), s > 0 ? 1u : 0u);
+  };
+  auto issue_i1 = [&]() {
+#pragma unroll 1
+    for (int T = 0; T < 8; ++T)
+#pragma unroll 1
+      for (int s = 0; s < 2; ++s)
+        g_mma(tmem + 16u * T, g_desc(aA + T * kI1Tile + s * 2 * kI1Lbo, kI1Lbo, kI1Sbo),
+              g_desc(aB + kBI1 + s * 256, 128, 512), g_idesc(16), s > 0 ? 1u : 0u);
+  };
+
+  const int Bh = B >> 1;
+  // Between stages a thread keeps, for its 32 times t = l + 128 w + 32 i + 1024 n3,
+  // the bf16 pair (item b, item b + 1) that multiplies the stage output: the
+  // input v before stage 0, the gate x_n after stage n; the convolution itself
+  // stays in TMEM (the output of I1) and is read again where it is needed.
+  uint32_t zp[4][8];
+  float u = 0.f;   // unscale factor of the I1 output
+  // z row i of the current stage input (stage 0: v; later: I1 output * u * gate)
+  auto z_row = [&](int i, bool first, float2 (&zz)[8]) {
+    if (first) {
+#pragma unroll
+      for (int n3 = 0; n3 < 8; ++n3)
+        zz[n3] = make_float2(__uint_as_float(zp[i][n3] << 16), __uint_as_float(zp[i][n3] & 0xffff0000u));
+    } else {
+      uint32_t r[16];
+      g_ld16(tlane + 16u * (2 * i + hw), r);
+      g_ld_wait();
+#pragma unroll
+      for (int n3 = 0; n3 < 8; ++n3)
+        zz[n3] = make_float2(__uint_as_float(r[2 * n3]) * (u * __uint_as_float(zp[i][n3] << 16)),
+                             __uint_as_float(r[2 * n3 + 1]) * (u * __uint_as_float(zp[i][n3] & 0xffff0000u)));
+    }
+  };
+  // bf16 pairs of rows r0, r1 at this thread's 32 times
+  auto load_pairs = [&](const __nv_bfloat16* base, size_t r0, size_t r1, size_t tb) {
+    const unsigned short* g0p = reinterpret_cast<const unsigned short*>(base + r0 + tb);
+    const unsigned short* g1p = reinterpret_cast<const unsigned short*>(base + r1 + tb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int n3 = 0; n3 < 8; ++n3)
+        zp[i][n3] = (uint32_t)__ldcs(g0p + 32 * i + 1024 * n3) | ((uint32_t)__ldcs(g1p + 32 * i + 1024 * n3) << 16);
+  };
+  for (long long p = blockIdx.x; p < npairs; p += gridDim.x) {
+    const int c = (int)(p / Bh);
+    const int b0 = 2 * (int)(p % Bh);
+    const size_t r0 = ((size_t)b0 * D + c) * (size_t)kGL;
+    const size_t r1 = r0 + (size_t)D * kGL;
+    const size_t tb = (size_t)(l + 128 * w);
+    load_pairs(v, r0, r1, tb);
+
+    for (int n = 0; n < N; ++n) {
+      const unsigned char* hrow = hptr[n] + (size_t)c * kGHRowBytes;
+      const uint32_t* hw32 = reinterpret_cast<const uint32_t*>(hrow);
+      const float inv_fc = __ldg(reinterpret_cast<const float*>(hrow + 4 * kGP));
+      // ---- input scale: CTA max |component| of z
+      float zm = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 zz[8];
+        z_row(i, n == 0, zz);
+#pragma unroll
+        for (int n3 = 0; n3 < 8; ++n3) zm = fmaxf(zm, fmaxf(fabsf(zz[n3].x), fabsf(zz[n3].y)));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zm = fmaxf(zm, __shfl_xor_sync(0xffffffffu, zm, o));
+      if (l == 0) red[w] = zm;
+      __syncthreads();
+      zm = red[0];
+#pragma unroll
+      for (int k = 1; k < 8; ++k) zm = fmaxf(zm, red[k]);
+      float s_in, inv_s;
+      g_scale_in(zm, s_in, inv_s);
+      // ---- F1 operand: own rows, K = n3 < 8
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 zz[8];
+        z_row(i, n == 0, zz);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint4 q4;
+          q4.x = g_pack(zz[4 * cc].x * s_in, zz[4 * cc].y * s_in);
+          q4.y = g_pack(zz[4 * cc + 1].x * s_in, zz[4 * cc + 1].y * s_in);
+          q4.z = g_pack(zz[4 * cc + 2].x * s_in, zz[4 * cc + 2].y * s_in);
+          q4.w = g_pack(zz[4 * cc + 3].x * s_in, zz[4 * cc + 3].y * s_in);
+          *reinterpret_cast<uint4*>(sA + f1_base + cc * 128 + i * 8192) = q4;
+        }
+      }
+      if (!level(issue_f1)) goto done;
+      // ---- F1 out: twiddle w_P^{m' k3}, to F2 rows (k3, m'' = l) at K = 4w + i
+      {
+        float2 cur[4], tw1i[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          cur[i] = make_float2(1.f, 0.f);
+          // w_512^i, i < 4
+          const float2 w512 = i == 0 ? make_float2(1.f, 0.f)
+                              : i == 1 ? make_float2(0.99992470183914454f, -0.01227153828571993f)
+                              : i == 2 ? make_float2(0.99969881869620425f, -0.02454122852291229f)
+                                       : make_float2(0.99932238458834954f, -0.03680722294135883f);
+          tw1i[i] = g_cmul(g_opaque(tw1), w512);
+        }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {   // k3 = 8 hf .. 8 hf + 7
+          uint32_t pk[4][8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t r[16];
+            g_ld16(tlane + 32u * (2 * i + hw) + 16u * hf, r);
+            g_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float2 vv = g_cmul(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), cur[i]);
+              pk[i][j] = g_pack(vv.x, vv.y);
+              cur[i] = g_cmul(cur[i], tw1i[i]);
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(sA + f12_base + 4096 * (8 * hf + j)) =
+                make_uint4(pk[0][j], pk[1][j], pk[2][j], pk[3][j]);
+        }
+      }
+      if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBF32); })) goto done;
+      // ---- F2 out: twiddle w_1024^{m'' k2}, to F3 rows (k3, k2) at K = m'' = l
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const float2 twb = g_opaque(tw2);
+        float2 cur = make_float2(1.f, 0.f);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[32];
+          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
+          g_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int k2 = 16 * hf + j;
+            const float2 vv = g_cmul(g_cval(r, j), cur);
+            const uint32_t off = (uint32_t)(2 * (k2 >> 4) * kF3Tile + (k2 & 3) * 16 + 512 * ((k2 >> 2) & 3));
+            *reinterpret_cast<uint32_t*>(sA + (f23_base + t * f23_step) + off) = g_pack(vv.x, vv.y);
+            cur = g_cmul(cur, twb);
+          }
+        }
+      }
+      if (!level([&]() { issue_c(kF3Tile, kF3Lbo, kF3Sbo, kBF32); })) goto done;
+      // ---- F3 out: C[k3 + 16 k2 + 512 k1] times the spectrum copy, times 2^-30;
+      // own rows as the I3 operand (K = k1)
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const int r3 = 128 * (hw + 2 * t) + 32 * q + l;
+        const uint4* hp = reinterpret_cast<const uint4*>(hw32 + (size_t)r3 * 32);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint4 hv[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) hv[k] = __ldcs(hp + 4 * hf + k);
+          uint32_t r[32];
+          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
+          g_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t hu[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 hf2 = __half22float2(*reinterpret_cast<const __half2*>(&hu[e]));
+              const float2 cv = g_cval(r, 4 * k + e);
+              const float2 yv = g_cmul(make_float2(cv.x * 0x1p-30f, cv.y * 0x1p-30f), hf2);
+              o[e] = g_pack(yv.x, yv.y);
+            }
+            *reinterpret_cast<uint4*>(sA + (i3_base + t * i3_step) + (4 * hf + k) * 128) = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
+      }
+      if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBI32); })) goto done;
+      // ---- I3 out: twiddle w_1024^{-m'' k2}, to I2 rows (k3, m'') at K = k2
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        const float2 tw3 = g_opaque(t ? tw3b : tw3a);
+        float2 cur = make_float2(1.f, 0.f);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[32];
+          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
+          g_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int mpp = 16 * hf + j;
+            const float2 vv = g_cmul(g_cval(r, j), cur);
+            const uint32_t off = (uint32_t)((16 * (mpp >> 3) + 2 * (mpp & 1) + 4 * ((mpp >> 1) & 3)) * 1024);
+            *reinterpret_cast<uint32_t*>(sA + (i32_base + t * i32_step) + off) = g_pack(vv.x, vv.y);
+            cur = g_cmul(cur, tw3);
+          }
+        }
+      }
+      if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBI32); })) goto done;
+      // ---- I2 out: twiddle w_P^{-(m'' + 32 n2) k3}, to I1 rows m' at K = k3
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+        float2 cur = g_opaque(t ? st2b : st2a);
+        const float2 twb = g_opaque(tw2i);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[32];
+          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
+          g_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n2 = 16 * hf + j;
+            const float2 vv = g_cmul(g_cval(r, j), cur);
+            const int jj = n2 >> 2, ii = n2 & 3;
+            const uint32_t off = (uint32_t)((2 * ii + (jj >> 2)) * kI1Tile + 512 * (jj & 3));
+            *reinterpret_cast<uint32_t*>(sA + (i21_base + t * i21_step) + off) = g_pack(vv.x, vv.y);
+            cur = g_cmul(cur, twb);
+          }
+        }
+      }
+      // gate rows of this stage, loaded while the last level runs
+      load_pairs(xptr[n], r0, r1, tb);
+      if (!level(issue_i1)) goto done;
+      u = 0x1p16f * inv_s * inv_fc;
+    }
+    // ---- y: the last stage's I1 output, unscaled and gated
+    {
+      __nv_bfloat16* y0 = y + r0 + tb;
+      __nv_bfloat16* y1 = y + r1 + tb;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 zz[8];
+        z_row(i, false, zz);
+#pragma unroll
+        for (int n3 = 0; n3 < 8; ++n3) {
+          y0[32 * i + 1024 * n3] = __float2bfloat16_rn(zz[n3].x);
+          y1[32 * i + 1024 * n3] = __float2bfloat16_rn(zz[n3].y);
+        }
+      }
+    }
+    // the next pair's first level overwrites TMEM: order these reads before it
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  }
+done:
+  // after a timeout: wait (bounded, 1 s) for the MMAs of the last issued level
+  if (!ok) g_wait(abar, phase ^ 1, 1000000000ull);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGCols));
+}
+
+// Spectrum copy for tcg_forward_kernel, one CTA per channel: 2L f16x2 bins of
+// f_c H[k] in F3-row order (word r * 32 + k1 for row r = (k3, k2) and bin
+// k = k3 + 16 k2 + 512 k1, H the 2L-point spectrum of the zero-padded filter),
+// then 1 / f_c. The natural copy holds H / (4L) for k < L, bin 0 packing
+// (H[0], H[L]); bins above L are conjugate mirrors. f_c is the power of two
+// that brings the largest component of f_c H into [2^14, 2^15).
+__global__ void tcg_spectrum_kernel(const float2* __restrict__ nat, unsigned char* __restrict__ out) {
+  __shared__ float redm[8];
+  const int c = blockIdx.x, tid = threadIdx.x;
+  const float2* __restrict__ nr = nat + (size_t)c * kGL;
+  unsigned char* row = out + (size_t)c * kGHRowBytes;
+  float mx = 0.f;
+  for (int i = tid; i < kGL; i += blockDim.x) mx = fmaxf(mx, fmaxf(fabsf(nr[i].x), fabsf(nr[i].y)));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) redm[tid >> 5] = mx;
+  __syncthreads();
+  mx = redm[0];
+  for (int k = 1; k < (int)(blockDim.x >> 5); ++k) mx = fmaxf(mx, redm[k]);
+  mx *= (float)(2 * kGP);                                        // largest component of H
+  int e = (int)((__float_as_uint(mx) >> 23) & 0xff);             // mx < 2^(e - 126)
+  e = e < 15 ? 15 : (e > 254 ? 254 : e);
+  const float fH = __uint_as_float((unsigned)(268 - e > 254 ? 254 : 268 - e) << 23);   // 2^(141 - e)
+  float inv_f = __uint_as_float((unsigned)(e - 14) << 23);                              // 2^(e - 141)
+  float f = fH * (float)(2 * kGP);                               // applied to the natural copy
+  if (mx == 0.f) { f = 1.f; inv_f = 1.f; }
+  uint32_t* wds = reinterpret_cast<uint32_t*>(row);
+  for (int idx = tid; idx < kGP; idx += blockDim.x) {
+    const int r = idx >> 5, k1 = idx & 31;
+    const int T = r >> 7, p = r & 127;
+    // row r = 128 T + p of F3: k3 = 8 (T & 1) + ((p >> 2) & 7), k2 = (p & 3) + 4 (p >> 5) + 16 (T >> 1)
+    const int k3 = 8 * (T & 1) + ((p >> 2) & 7);
+    const int k2 = (p & 3) + 4 * (p >> 5) + 16 * (T >> 1);
+    const int k = k3 + 16 * k2 + 512 * k1;
+    float2 hv;
+    if (k == 0) hv = make_float2(nr[0].x, 0.f);
+    else if (k == kGL) hv = make_float2(nr[0].y, 0.f);
+    else if (k < kGL) hv = nr[k];
+    else { const float2 m = nr[kGP - k]; hv = make_float2(m.x, -m.y); }
+    wds[idx] = g_pack(f * hv.x, f * hv.y);
+  }
+  if (tid == 0) {
+    float* tail = reinterpret_cast<float*>(row + 4 * kGP);
+    tail[0] = inv_f;
+    tail[1] = 0.f;
+    tail[2] = 0.f;
+    tail[3] = 0.f;
+  }
+}
+
+cudaError_t launch_tcg_forward(const FusedLaunch& p, cudaStream_t s) {
+  auto k = tcg_forward_kernel;
+  cudaError_t e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute((const void*)k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  // Two CTAs per SM: shared memory admits at most two, and their TMEM
+  // allocations (256 columns each) fill the SM's 512 columns exactly, so no
+  // allocation ever waits on another CTA.
+  static_assert(2 * kGCols <= 512 && 3 * (kGSmem + 1024) > 228 * 1024, "at most two resident CTAs per SM");
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  int grid = 2 * sms;
+  const long long npairs = (long long)(p.B / 2) * p.D;
+  if ((long long)grid > npairs) grid = (int)npairs;
+  GatePtrs<__nv_bfloat16> xp;
+  for (int i = 0; i < kMaxOrder; ++i) xp.p[i] = reinterpret_cast<const __nv_bfloat16*>(p.x[i]);
+  k<<<grid, kGT, kGSmem, s>>>(reinterpret_cast<const __nv_bfloat16*>(p.v), xp, p.hh,
+                              reinterpret_cast<__nv_bfloat16*>(p.y), p.B, p.D, p.N, npairs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tcg_spectrum(const float2* nat, float2* tcs, int D, cudaStream_t s) {
+  tcg_spectrum_kernel<<<D, 256, 0, s>>>(nat, reinterpret_cast<unsigned char*>(tcs));
+  return cudaGetLastError();
+}
+
+int tcg_read_and_clear_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tcg_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_tcg_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
+}  // namespace hyena

@@ -29,8 +29,12 @@
  *    rejected call launches nothing. HYENA_ERR_CUDA reports a launch error
  *    (see hyena_last_cuda_error()).
  *  - Activations v, x_n, y are row-major [B][D][L] (time fastest) in the
- *    storage type `dtype`; the arithmetic is float32 throughout and bf16
- *    results are rounded to nearest even.
+ *    storage type `dtype`; bf16 results are rounded to nearest even. The
+ *    arithmetic is float32, except that hyena_forward with bf16 I/O, B even
+ *    and L in {1024, 2048, 8192} runs its transforms on the tensor cores with
+ *    f16 operands (scaled by exact powers of two) and float32 accumulation;
+ *    that adds an error below the bf16 output rounding (relative L2 within
+ *    the bf16 tolerance of 8e-3).
  *  - For the 1-D FFT calls L must be a power of two with 16 <= L <= 2^20
  *    (HYENA_ERR_UNSUPPORTED otherwise); 1 <= N <= 8; B, D >= 1. The
  *    StripedHyena calls take any L >= 1 and the HyenaND calls state their
@@ -335,16 +339,18 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
                                       hyena_stream stream);
 
 /*
- * Kernels that wait on mbarriers for asynchronous copies (the striped
- * bulk-copy kernel of hyena_striped_forward, taken when a row's byte length
- * is a multiple of 16) bound every wait in time: a wait gives up 0.2 s of
- * GPU global time after it started (each polling step suspends for at most
- * 20 us). A wait that runs out makes every thread block of that launch stop
- * early (its outputs are then invalid) and sets a sticky flag on the current
- * device; before exiting, such a block waits at most 1 s more for the copies
- * it still has in flight. This call synchronises with the device, reads and
- * clears the flag: HYENA_OK if no wait ran out since the last call,
- * HYENA_ERR_TIMEOUT otherwise (HYENA_ERR_CUDA if it cannot be read).
+ * Kernels that wait on mbarriers for asynchronous copies or tensor-core
+ * completions (the striped bulk-copy kernel of hyena_striped_forward, taken
+ * when a row's byte length is a multiple of 16, and the tcgen05 forward of
+ * hyena_forward for bf16, B even, L = 8192) bound every wait in time: a
+ * wait gives up 0.2 s of GPU global time after it started (each polling
+ * step suspends for at most 20 us). A wait that runs out makes every thread
+ * block of that launch stop early (its outputs are then invalid) and sets a
+ * sticky flag on the current device; before exiting, such a block waits at
+ * most 1 s more for the copies or tensor-core work it still has in flight.
+ * This call synchronises with the device, reads and clears the flag:
+ * HYENA_OK if no wait ran out since the last call, HYENA_ERR_TIMEOUT
+ * otherwise (HYENA_ERR_CUDA if it cannot be read).
  */
 hyena_status hyena_device_timeouts(void);
 

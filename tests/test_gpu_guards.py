@@ -91,6 +91,7 @@ def run_guarded(hy, w, fill, f16=False):
     (2, "f32", 1, 3, 1024, False),       # fused SIMT
     (2, "bf16", 2, 3, 2048, False),      # tensor-core fused
     (3, "bf16", 3, 2, 8192, False),      # fused SIMT, staged spectra
+    (3, "bf16", 2, 3, 8192, False),      # tcgen05 GEMM levels
     (2, "f32", 2, 2, 16384, False),      # fused SIMT, 1024 threads per channel
     (2, "bf16", 1, 3, 32768, False),     # four-step
     (2, "bf16", 1, 5, 131072, False),    # four-step, rows of 1024

@@ -111,13 +111,14 @@ SWEEP = [
     (2, "bf16", 6, 3, 2048),
     # odd B at a tensor-core length falls back to the SIMT kernel
     (2, "bf16", 3, 2, 2048),
-    # tensor-core four-step: bf16, 2^16 <= L <= 2^20 (rows of R * 256 points, R = 1 .. 16)
+    # tcgen05 GEMM-level kernel: bf16, even B, L = 8192 (more in test_gpu_tcgen05.py)
+    (3, "bf16", 2, 2, 8192),
+    # four-step, bf16, 2^16 <= L <= 2^20 (rows of 1024 or 4096 points)
     (1, "bf16", 1, 2, 65536),
     (2, "bf16", 2, 3, 131072),
     (3, "bf16", 1, 2, 262144),
     (3, "bf16", 3, 1, 524288),
     (2, "bf16", 1, 2, 1048576),
-    # order 4 keeps the float32 four-step kernels at these lengths
     (4, "bf16", 3, 1, 524288),
 ]
 
@@ -132,7 +133,7 @@ def test_forward_shapes(hy, N, dtype, B, D, L):
     assert err.max() <= TOL[dtype], err.max()
 
 
-@pytest.mark.parametrize("L,dtype", [(2048, "f32"), (2048, "bf16"), (32768, "f32"), (131072, "bf16")])
+@pytest.mark.parametrize("L,dtype", [(2048, "f32"), (2048, "bf16"), (8192, "bf16"), (32768, "f32"), (131072, "bf16")])
 def test_forward_in_place_and_waves(hy, L, dtype):
     import torch
     w = synth.custom(2, dtype, 2, 3, L, seed=5)
