@@ -98,7 +98,7 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     p.B = B; p.D = D; p.L = ly.L; p.N = N;
     p.bf16 = bf16;
     p.spec16 = spec16;
-    if (allow_tc && has_tc_copy(ly) && p.bf16 && (B % 2) == 0) {
+    if (allow_tc && p.bf16 && (B % 2) == 0 && (ly.tc || (ly.tcg && N <= kTcgMaxOrder))) {
       // tensor-core kernel on pairs of batch items, reading the tensor-core copy of the spectra
       for (int n = 0; n < N; ++n)
         p.hh.p[n] = reinterpret_cast<const float2*>(hhat[n]) + tc_spectrum_offset(ly, D);

@@ -41,8 +41,12 @@ struct Layout {
 // Lengths with a tensor-core forward (outer radix R0 = L / 128 in {8, 16}).
 constexpr int kTcMinL = 1024;
 constexpr int kTcMaxL = 2048;
-// Length of the tcgen05 GEMM-level forward.
+// Length of the tcgen05 GEMM-level forward, and the highest order it serves:
+// its f16 operands add an error that compounds through the gates, within the
+// bf16 tolerance up to order 3 (float64 model of its scalings: 3.1e-3 at order
+// 3, 6.1e-3 at order 4 and 1.3e-2 at order 8 on seeded N(0,1) gates).
 constexpr int kTcgL = 8192;
+constexpr int kTcgMaxOrder = 3;
 
 inline int ilog2_exact(int v) {
   int l = 0;

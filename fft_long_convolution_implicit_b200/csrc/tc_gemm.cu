@@ -29,10 +29,12 @@
 // between the N stages. One thread issues the MMAs; completion arrives on an
 // mbarrier through tcgen05.commit; every wait is bounded in time.
 //
-// Scaling (exact powers of two): z is scaled so max |component| < 2^6, which
-// keeps every f16 operand of F1..F3 below 2^15; the spectrum copy is scaled per
-// channel to [2^14, 2^15) and the product by 2^-30, which keeps I3..I1 below
-// 2^15; all factors are removed at the gate.
+// Scaling (exact powers of two): z is scaled so max |component| < 2^6; the
+// DFT matrices carry 2^-4 (F1), 2^-8 (F2, F3) and 2^-5 (I3, I2), which keeps
+// every f16 operand below 2^15 for any input (each level grows a bound by at
+// most its length) while every nonzero matrix entry stays an f16 normal; the
+// spectrum copy is scaled per channel to [2^14, 2^15). All factors (2^-30 in
+// all) are removed at the gate.
 #include <cuda_fp16.h>
 
 #include "fft_engine.cuh"
@@ -92,15 +94,23 @@ __device__ __forceinline__ void g_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, multiple of 16 bytes).
+__device__ __forceinline__ void g_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ unsigned long long g_globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
-// Wait for an mbarrier phase, bounded in time (each try suspends at most
-// 20 us; false once limit_ns of global time have passed).
+// Wait for an mbarrier phase, bounded in time (each try suspends for at most
+// HYENA_TCG_SUSPEND_NS; false once limit_ns of global time have passed).
 constexpr unsigned long long kGWaitLimitNs = 200000000ull;   // 0.2 s
+#ifndef HYENA_TCG_SUSPEND_NS
+#define HYENA_TCG_SUSPEND_NS 20000
+#endif
 __device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t phase, unsigned long long limit_ns = kGWaitLimitNs) {
   const unsigned long long t0 = g_globaltimer_ns();
   for (;;) {
@@ -109,7 +119,7 @@ __device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t phase, unsigned lo
         "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, P1;\n\t}\n"
         : "=r"(done)
-        : "r"(bar), "r"(phase), "r"(20000u)
+        : "r"(bar), "r"(phase), "r"((uint32_t)HYENA_TCG_SUSPEND_NS)
         : "memory");
     if (done) return true;
     if (g_globaltimer_ns() - t0 > limit_ns) return false;
@@ -135,7 +145,19 @@ __device__ __forceinline__ void g_ld16(uint32_t addr, uint32_t (&r)[16]) {
       : G_LD_REGS16(r, 0)
       : "r"(addr));
 }
-__device__ __forceinline__ void g_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's TMEM loads. The loaded registers are operands of the
+// wait, so no use of them can be scheduled before it.
+#define G_RW_REGS16(r, o)                                                                                      \
+  "+r"(r[o + 0]), "+r"(r[o + 1]), "+r"(r[o + 2]), "+r"(r[o + 3]), "+r"(r[o + 4]), "+r"(r[o + 5]),              \
+      "+r"(r[o + 6]), "+r"(r[o + 7]), "+r"(r[o + 8]), "+r"(r[o + 9]), "+r"(r[o + 10]), "+r"(r[o + 11]),        \
+      "+r"(r[o + 12]), "+r"(r[o + 13]), "+r"(r[o + 14]), "+r"(r[o + 15])
+__device__ __forceinline__ void g_wait32(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : G_RW_REGS16(r, 0), G_RW_REGS16(r, 16)::"memory");
+}
+__device__ __forceinline__ void g_wait16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : G_RW_REGS16(r, 0)::"memory");
+}
+#undef G_RW_REGS16
 #undef G_LD_REGS16
 
 __device__ __forceinline__ uint32_t g_pack(float re, float im) {
@@ -143,10 +165,9 @@ __device__ __forceinline__ uint32_t g_pack(float re, float im) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// a * b with packed f32x2 arithmetic: (a.x b.x - a.y b.y, a.x b.y + a.y b.x)
+// a * b: (a.x b.x - a.y b.y, a.x b.y + a.y b.x), two FMUL and two FFMA
 __device__ __forceinline__ float2 g_cmul(float2 a, float2 b) {
-  const float2 t = __fmul2_rn(make_float2(a.y, a.y), make_float2(-b.y, b.x));
-  return __ffma2_rn(make_float2(a.x, a.x), b, t);
+  return make_float2(fmaf(a.x, b.x, -(a.y * b.y)), fmaf(a.x, b.y, a.y * b.x));
 }
 
 // The twiddle powers of a recurrence depend only on per-thread constants; a
@@ -159,8 +180,34 @@ __device__ __forceinline__ float2 g_opaque(float2 a) {
   return b;
 }
 
-__device__ __forceinline__ float2 g_cval(const uint32_t (&r)[32], int j) {
+template <int R>
+__device__ __forceinline__ float2 g_cval(const uint32_t (&r)[R], int j) {
   return make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+}
+
+// Four TMEM chunks of C columns (C = 16 or 32) read one ahead of their use:
+// chunk j + 1 is loading while chunk j is processed.
+template <int C, typename Addr, typename Proc>
+__device__ __forceinline__ void g_pipe4(Addr addr, Proc proc) {
+  uint32_t ra[C], rb[C];
+  auto ld = [](uint32_t a, uint32_t (&r)[C]) {
+    if constexpr (C == 32) g_ld32(a, r); else g_ld16(a, r);
+  };
+  auto wt = [](uint32_t (&r)[C]) {
+    if constexpr (C == 32) g_wait32(r); else g_wait16(r);
+  };
+  ld(addr(0), ra);
+  wt(ra);
+  ld(addr(1), rb);
+  proc(0, ra);
+  wt(rb);
+  ld(addr(2), ra);
+  proc(1, rb);
+  wt(ra);
+  ld(addr(3), rb);
+  proc(2, ra);
+  wt(rb);
+  proc(3, rb);
 }
 
 // w_n^{e} = exp(-2 pi i e / n) for an exact integer e (|e| < n)
@@ -187,15 +234,19 @@ __device__ __forceinline__ void g_put(unsigned char* sB, uint32_t base, int K, i
   *reinterpret_cast<__half*>(sB + o) = __float2half_rn(v);
 }
 
-// Real form of F[o][i] = w_n^{sign o i} (outputs o < no, inputs i < ni) at `base`:
-// rows 2o + rho, columns 2i + sigma: [[Fr, -Fi], [Fi, Fr]].
-__device__ void g_build_dft(unsigned char* sB, uint32_t base, int n, int no, int ni, bool inverse, int tid) {
+// Real form of scale * F[o][i], F[o][i] = w_n^{sign o i} (outputs o < no,
+// inputs i < ni) at `base`: rows 2o + rho, columns 2i + sigma: [[Fr, -Fi], [Fi, Fr]].
+// scale is a power of two small enough to keep every nonzero entry an f16 normal.
+__device__ void g_build_dft(unsigned char* sB, uint32_t base, int n, int no, int ni, bool inverse, float scale,
+                            int tid) {
   const int K = 2 * ni;
   for (int idx = tid; idx < no * ni; idx += kGT) {
     const int o = idx / ni, i = idx % ni;
     const int e = (o * i) % n;
     float2 w = g_root(e, n);
     if (inverse) w.y = -w.y;
+    w.x *= scale;
+    w.y *= scale;
     g_put(sB, base, K, 2 * o, 2 * i, w.x);
     g_put(sB, base, K, 2 * o, 2 * i + 1, -w.y);
     g_put(sB, base, K, 2 * o + 1, 2 * i, w.y);
@@ -232,10 +283,10 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(abar), "r"(1));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  g_build_dft(sB, kBF1, 16, 16, 8, false, tid);
-  g_build_dft(sB, kBF32, 32, 32, 32, false, tid);
-  g_build_dft(sB, kBI32, 32, 32, 32, true, tid);
-  g_build_dft(sB, kBI1, 16, 8, 16, true, tid);
+  g_build_dft(sB, kBF1, 16, 16, 8, false, 0x1p-4f, tid);
+  g_build_dft(sB, kBF32, 32, 32, 32, false, 0x1p-8f, tid);
+  g_build_dft(sB, kBI32, 32, 32, 32, true, 0x1p-5f, tid);
+  g_build_dft(sB, kBI1, 16, 8, 16, true, 1.f, tid);
 
   // ---- per-thread row ownership, twiddle bases and store addresses
   // F1 / I1 rows i: m' = l + 128 w + 32 i (tile 2i + hw); time t = m' + 1024 n3
@@ -290,26 +341,30 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     return true;
   };
+  // MMA issue (thread 0): the start-address field of a descriptor is its low
+  // 14 bits (address / 16), so a base descriptor plus offset / 16 addresses
+  // every tile and K step (all offsets stay inside shared memory).
   auto issue_f1 = [&]() {
-#pragma unroll 1
-    for (int T = 0; T < 8; ++T)
-      g_mma(tmem + 32u * T, g_desc(aA + T * kF1Tile, kF1Lbo, kF1Sbo), g_desc(aB + kBF1, 128, 256), g_idesc(32), 0u);
+    const uint64_t da = g_desc(aA, kF1Lbo, kF1Sbo), db = g_desc(aB + kBF1, 128, 256);
+#pragma unroll
+    for (int T = 0; T < 8; ++T) g_mma(tmem + 32u * T, da + (T * kF1Tile >> 4), db, g_idesc(32), 0u);
   };
   auto issue_c = [&](uint32_t tile, uint32_t lbo, uint32_t sbo, uint32_t bmat) {
-#pragma unroll 1
+    const uint64_t da = g_desc(aA, lbo, sbo), db = g_desc(aB + bmat, 128, 1024);
+#pragma unroll
     for (int T = 0; T < 4; ++T)
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < 4; ++s)
-        g_mma(tmem + 64u * T, g_desc(aA + T * tile + s * 2 * lbo, lbo, sbo), g_desc(aB + bmat + s * 256, 128, 1024),
-              g_idesc(64), s > 0 ? 1u : 0u);
+        g_mma(tmem + 64u * T, da + ((T * tile + s * 2 * lbo) >> 4), db + (s * 256 >> 4), g_idesc(64), s > 0 ? 1u : 0u);
   };
   auto issue_i1 = [&]() {
-#pragma unroll 1
+    const uint64_t da = g_desc(aA, kI1Lbo, kI1Sbo), db = g_desc(aB + kBI1, 128, 512);
+#pragma unroll
     for (int T = 0; T < 8; ++T)
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < 2; ++s)
-        g_mma(tmem + 16u * T, g_desc(aA + T * kI1Tile + s * 2 * kI1Lbo, kI1Lbo, kI1Sbo),
-              g_desc(aB + kBI1 + s * 256, 128, 512), g_idesc(16), s > 0 ? 1u : 0u);
+        g_mma(tmem + 16u * T, da + ((T * kI1Tile + s * 2 * kI1Lbo) >> 4), db + (s * 256 >> 4), g_idesc(16),
+              s > 0 ? 1u : 0u);
   };
 
   const int Bh = B >> 1;
@@ -319,22 +374,19 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
   // stays in TMEM (the output of I1) and is read again where it is needed.
   uint32_t zp[4][8];
   float u = 0.f;   // unscale factor of the I1 output
-  // z row i of the current stage input (stage 0: v; later: I1 output * u * gate)
-  auto z_row = [&](int i, bool first, float2 (&zz)[8]) {
-    if (first) {
+  // z of row i (8 values n3) from the I1 output r (or from v before stage 0)
+  // z of row i (8 values n3) times `scale`: I1 output r times (u * scale) times
+  // the gate pair, or (before stage 0) the input pair times scale
+  auto z_of = [&](int i, const uint32_t (&r)[16], bool first, float scale, float2 (&zz)[8]) {
+    const float us = first ? scale : u * scale;
 #pragma unroll
-      for (int n3 = 0; n3 < 8; ++n3)
-        zz[n3] = make_float2(__uint_as_float(zp[i][n3] << 16), __uint_as_float(zp[i][n3] & 0xffff0000u));
-    } else {
-      uint32_t r[16];
-      g_ld16(tlane + 16u * (2 * i + hw), r);
-      g_ld_wait();
-#pragma unroll
-      for (int n3 = 0; n3 < 8; ++n3)
-        zz[n3] = make_float2(__uint_as_float(r[2 * n3]) * (u * __uint_as_float(zp[i][n3] << 16)),
-                             __uint_as_float(r[2 * n3 + 1]) * (u * __uint_as_float(zp[i][n3] & 0xffff0000u)));
+    for (int n3 = 0; n3 < 8; ++n3) {
+      const float g0 = __uint_as_float(zp[i][n3] << 16) * us, g1 = __uint_as_float(zp[i][n3] & 0xffff0000u) * us;
+      zz[n3] = first ? make_float2(g0, g1)
+                     : make_float2(__uint_as_float(r[2 * n3]) * g0, __uint_as_float(r[2 * n3 + 1]) * g1);
     }
   };
+  auto i1_addr = [&](int i) { return tlane + 16u * (2 * i + hw); };
   // bf16 pairs of rows r0, r1 at this thread's 32 times
   auto load_pairs = [&](const __nv_bfloat16* base, size_t r0, size_t r1, size_t tb) {
     const unsigned short* g0p = reinterpret_cast<const unsigned short*>(base + r0 + tb);
@@ -357,14 +409,37 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
       const unsigned char* hrow = hptr[n] + (size_t)c * kGHRowBytes;
       const uint32_t* hw32 = reinterpret_cast<const uint32_t*>(hrow);
       const float inv_fc = __ldg(reinterpret_cast<const float*>(hrow + 4 * kGP));
+      // L2 prefetch (bulk, no shared-memory destination) of what this stage
+      // reads from HBM later: its spectrum row, its gate rows, and after the
+      // last stage the next pair's input rows
+      if (tid == 0) {
+        g_prefetch_l2(hrow, (uint32_t)kGHRowBytes);
+        g_prefetch_l2(xptr[n] + r0, 2 * kGL);
+        g_prefetch_l2(xptr[n] + r1, 2 * kGL);
+        if (n + 1 == N && p + gridDim.x < npairs) {
+          const long long pn = p + gridDim.x;
+          const size_t q0 = ((size_t)(2 * (int)(pn % Bh)) * D + (size_t)(pn / Bh)) * (size_t)kGL;
+          g_prefetch_l2(v + q0, 2 * kGL);
+          g_prefetch_l2(v + q0 + (size_t)D * kGL, 2 * kGL);
+        }
+      }
+      const bool first = (n == 0);
       // ---- input scale: CTA max |component| of z
       float zm = 0.f;
+      {
+        auto proc = [&](int i, const uint32_t (&r)[16]) {
+          float2 zz[8];
+          z_of(i, r, first, 1.f, zz);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 zz[8];
-        z_row(i, n == 0, zz);
+          for (int n3 = 0; n3 < 8; ++n3) zm = fmaxf(zm, fmaxf(fabsf(zz[n3].x), fabsf(zz[n3].y)));
+        };
+        if (first) {
+          uint32_t r[16];
 #pragma unroll
-        for (int n3 = 0; n3 < 8; ++n3) zm = fmaxf(zm, fmaxf(fabsf(zz[n3].x), fabsf(zz[n3].y)));
+          for (int i = 0; i < 4; ++i) proc(i, r);
+        } else {
+          g_pipe4<16>(i1_addr, proc);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) zm = fmaxf(zm, __shfl_xor_sync(0xffffffffu, zm, o));
@@ -376,22 +451,32 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
       float s_in, inv_s;
       g_scale_in(zm, s_in, inv_s);
       // ---- F1 operand: own rows, K = n3 < 8
+      {
+        auto proc = [&](int i, const uint32_t (&r)[16]) {
+          float2 zz[8];
+          z_of(i, r, first, s_in, zz);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float2 zz[8];
-        z_row(i, n == 0, zz);
+          for (int cc = 0; cc < 2; ++cc) {
+            uint4 q4;
+            q4.x = g_pack(zz[4 * cc].x, zz[4 * cc].y);
+            q4.y = g_pack(zz[4 * cc + 1].x, zz[4 * cc + 1].y);
+            q4.z = g_pack(zz[4 * cc + 2].x, zz[4 * cc + 2].y);
+            q4.w = g_pack(zz[4 * cc + 3].x, zz[4 * cc + 3].y);
+            *reinterpret_cast<uint4*>(sA + f1_base + cc * 128 + i * 8192) = q4;
+          }
+        };
+        if (first) {
+          uint32_t r[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint4 q4;
-          q4.x = g_pack(zz[4 * cc].x * s_in, zz[4 * cc].y * s_in);
-          q4.y = g_pack(zz[4 * cc + 1].x * s_in, zz[4 * cc + 1].y * s_in);
-          q4.z = g_pack(zz[4 * cc + 2].x * s_in, zz[4 * cc + 2].y * s_in);
-          q4.w = g_pack(zz[4 * cc + 3].x * s_in, zz[4 * cc + 3].y * s_in);
-          *reinterpret_cast<uint4*>(sA + f1_base + cc * 128 + i * 8192) = q4;
+          for (int i = 0; i < 4; ++i) proc(i, r);
+        } else {
+          g_pipe4<16>(i1_addr, proc);
         }
       }
       if (!level(issue_f1)) goto done;
-      // ---- F1 out: twiddle w_P^{m' k3}, to F2 rows (k3, m'' = l) at K = 4w + i
+      // ---- F1 out: twiddle w_P^{m' k3}, to F2 rows (k3, m'' = l) at K = 4w + i.
+      // Chunks: k3 half hf (8 outputs) of row i, the four rows of one half
+      // before the next; one 16-byte store per k3 gathers the four rows.
       {
         float2 cur[4], tw1i[4];
 #pragma unroll
@@ -405,20 +490,17 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
           tw1i[i] = g_cmul(g_opaque(tw1), w512);
         }
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {   // k3 = 8 hf .. 8 hf + 7
+        for (int hf = 0; hf < 2; ++hf) {
           uint32_t pk[4][8];
+          g_pipe4<16>([&](int i) { return tlane + 32u * (2 * i + hw) + 16u * hf; },
+                      [&](int i, const uint32_t (&r)[16]) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t r[16];
-            g_ld16(tlane + 32u * (2 * i + hw) + 16u * hf, r);
-            g_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float2 vv = g_cmul(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), cur[i]);
-              pk[i][j] = g_pack(vv.x, vv.y);
-              cur[i] = g_cmul(cur[i], tw1i[i]);
-            }
-          }
+                        for (int j = 0; j < 8; ++j) {
+                          const float2 vv = g_cmul(g_cval(r, j), cur[i]);
+                          pk[i][j] = g_pack(vv.x, vv.y);
+                          cur[i] = g_cmul(cur[i], tw1i[i]);
+                        }
+                      });
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             *reinterpret_cast<uint4*>(sA + f12_base + 4096 * (8 * hf + j)) =
@@ -426,98 +508,103 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
         }
       }
       if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBF32); })) goto done;
-      // ---- F2 out: twiddle w_1024^{m'' k2}, to F3 rows (k3, k2) at K = m'' = l
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
+      // ---- F2 out: twiddle w_1024^{m'' k2}, to F3 rows (k3, k2) at K = m'' = l.
+      // Chunk 2 t + hf: outputs k2 = 16 hf .. 16 hf + 15 of row t.
+      {
         const float2 twb = g_opaque(tw2);
         float2 cur = make_float2(1.f, 0.f);
+        g_pipe4<32>([&](int ch) { return tlane + 64u * (hw + 2 * (ch >> 1)) + 32u * (ch & 1); },
+                    [&](int ch, const uint32_t (&r)[32]) {
+                      const int t = ch >> 1, hf = ch & 1;
+                      if (hf == 0) cur = make_float2(1.f, 0.f);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
-          g_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int k2 = 16 * hf + j;
-            const float2 vv = g_cmul(g_cval(r, j), cur);
-            const uint32_t off = (uint32_t)(2 * (k2 >> 4) * kF3Tile + (k2 & 3) * 16 + 512 * ((k2 >> 2) & 3));
-            *reinterpret_cast<uint32_t*>(sA + (f23_base + t * f23_step) + off) = g_pack(vv.x, vv.y);
-            cur = g_cmul(cur, twb);
-          }
-        }
+                      for (int j = 0; j < 16; ++j) {
+                        const int k2 = 16 * hf + j;
+                        const float2 vv = g_cmul(g_cval(r, j), cur);
+                        cur = g_cmul(cur, twb);
+                        const uint32_t off =
+                            (uint32_t)(2 * (k2 >> 4) * kF3Tile + (k2 & 3) * 16 + 512 * ((k2 >> 2) & 3));
+                        *reinterpret_cast<uint32_t*>(sA + (f23_base + t * f23_step) + off) = g_pack(vv.x, vv.y);
+                      }
+                    });
       }
-      if (!level([&]() { issue_c(kF3Tile, kF3Lbo, kF3Sbo, kBF32); })) goto done;
-      // ---- F3 out: C[k3 + 16 k2 + 512 k1] times the spectrum copy, times 2^-30;
-      // own rows as the I3 operand (K = k1)
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        const int r3 = 128 * (hw + 2 * t) + 32 * q + l;
-        const uint4* hp = reinterpret_cast<const uint4*>(hw32 + (size_t)r3 * 32);
+      // ---- F3 out: 2^-20 C[k3 + 16 k2 + 512 k1] times the spectrum copy;
+      // own rows as the I3 operand (K = k1). Chunk 2 t + hf holds bins
+      // k1 = 16 hf .. 16 hf + 15 of row t; its 64 spectrum bytes are loaded
+      // one chunk ahead (the first before the level's wait).
+      {
+        const uint4* hp0 = reinterpret_cast<const uint4*>(hw32 + (size_t)(128 * hw + 32 * q + l) * 32);
+        constexpr int kRowStep = 256 * 32 / 4;   // uint4 from row t = 0 to row t = 1
+        uint4 hcur[4], hnext[4];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint4 hv[4];
+        for (int k = 0; k < 4; ++k) hcur[k] = __ldcs(hp0 + k);
+        if (!level([&]() { issue_c(kF3Tile, kF3Lbo, kF3Sbo, kBF32); })) goto done;
+        g_pipe4<32>([&](int ch) { return tlane + 64u * (hw + 2 * (ch >> 1)) + 32u * (ch & 1); },
+                    [&](int ch, const uint32_t (&r)[32]) {
+                      const int t = ch >> 1, hf = ch & 1;
+                      if (ch < 3) {
+                        const int tn = (ch + 1) >> 1, hn = (ch + 1) & 1;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) hv[k] = __ldcs(hp + 4 * hf + k);
-          uint32_t r[32];
-          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
-          g_ld_wait();
+                        for (int k = 0; k < 4; ++k) hnext[k] = __ldcs(hp0 + tn * kRowStep + 4 * hn + k);
+                      }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t hu[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
-            uint32_t o[4];
+                      for (int k = 0; k < 4; ++k) {
+                        const uint32_t hu[4] = {hcur[k].x, hcur[k].y, hcur[k].z, hcur[k].w};
+                        uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 hf2 = __half22float2(*reinterpret_cast<const __half2*>(&hu[e]));
-              const float2 cv = g_cval(r, 4 * k + e);
-              const float2 yv = g_cmul(make_float2(cv.x * 0x1p-30f, cv.y * 0x1p-30f), hf2);
-              o[e] = g_pack(yv.x, yv.y);
-            }
-            *reinterpret_cast<uint4*>(sA + (i3_base + t * i3_step) + (4 * hf + k) * 128) = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        }
+                        for (int e = 0; e < 4; ++e) {
+                          const float2 hf2 = __half22float2(*reinterpret_cast<const __half2*>(&hu[e]));
+                          const float2 cv = g_cval(r, 4 * k + e);
+                          const float2 yv = g_cmul(cv, hf2);
+                          o[e] = g_pack(yv.x, yv.y);
+                        }
+                        *reinterpret_cast<uint4*>(sA + (i3_base + t * i3_step) + (4 * hf + k) * 128) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                      }
+#pragma unroll
+                      for (int k = 0; k < 4; ++k) hcur[k] = hnext[k];
+                    });
       }
       if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBI32); })) goto done;
       // ---- I3 out: twiddle w_1024^{-m'' k2}, to I2 rows (k3, m'') at K = k2
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        const float2 tw3 = g_opaque(t ? tw3b : tw3a);
-        float2 cur = make_float2(1.f, 0.f);
+      {
+        float2 cur = make_float2(1.f, 0.f), twb = make_float2(1.f, 0.f);
+        g_pipe4<32>([&](int ch) { return tlane + 64u * (hw + 2 * (ch >> 1)) + 32u * (ch & 1); },
+                    [&](int ch, const uint32_t (&r)[32]) {
+                      const int t = ch >> 1, hf = ch & 1;
+                      if (hf == 0) {
+                        cur = make_float2(1.f, 0.f);
+                        twb = g_opaque(t ? tw3b : tw3a);
+                      }
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
-          g_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int mpp = 16 * hf + j;
-            const float2 vv = g_cmul(g_cval(r, j), cur);
-            const uint32_t off = (uint32_t)((16 * (mpp >> 3) + 2 * (mpp & 1) + 4 * ((mpp >> 1) & 3)) * 1024);
-            *reinterpret_cast<uint32_t*>(sA + (i32_base + t * i32_step) + off) = g_pack(vv.x, vv.y);
-            cur = g_cmul(cur, tw3);
-          }
-        }
+                      for (int j = 0; j < 16; ++j) {
+                        const int mpp = 16 * hf + j;
+                        const float2 vv = g_cmul(g_cval(r, j), cur);
+                        cur = g_cmul(cur, twb);
+                        const uint32_t off = (uint32_t)((16 * (mpp >> 3) + 2 * (mpp & 1) + 4 * ((mpp >> 1) & 3)) * 1024);
+                        *reinterpret_cast<uint32_t*>(sA + (i32_base + t * i32_step) + off) = g_pack(vv.x, vv.y);
+                      }
+                    });
       }
       if (!level([&]() { issue_c(kCTile, kCLbo, kCSbo, kBI32); })) goto done;
       // ---- I2 out: twiddle w_P^{-(m'' + 32 n2) k3}, to I1 rows m' at K = k3
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-        float2 cur = g_opaque(t ? st2b : st2a);
+      {
         const float2 twb = g_opaque(tw2i);
+        float2 cur = make_float2(1.f, 0.f);
+        g_pipe4<32>([&](int ch) { return tlane + 64u * (hw + 2 * (ch >> 1)) + 32u * (ch & 1); },
+                    [&](int ch, const uint32_t (&r)[32]) {
+                      const int t = ch >> 1, hf = ch & 1;
+                      if (hf == 0) cur = g_opaque(t ? st2b : st2a);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          g_ld32(tlane + 64u * (hw + 2 * t) + 32u * hf, r);
-          g_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n2 = 16 * hf + j;
-            const float2 vv = g_cmul(g_cval(r, j), cur);
-            const int jj = n2 >> 2, ii = n2 & 3;
-            const uint32_t off = (uint32_t)((2 * ii + (jj >> 2)) * kI1Tile + 512 * (jj & 3));
-            *reinterpret_cast<uint32_t*>(sA + (i21_base + t * i21_step) + off) = g_pack(vv.x, vv.y);
-            cur = g_cmul(cur, twb);
-          }
-        }
+                      for (int j = 0; j < 16; ++j) {
+                        const int n2 = 16 * hf + j;
+                        const float2 vv = g_cmul(g_cval(r, j), cur);
+                        const int jj = n2 >> 2, ii = n2 & 3;
+                        const uint32_t off = (uint32_t)((2 * ii + (jj >> 2)) * kI1Tile + 512 * (jj & 3));
+                        *reinterpret_cast<uint32_t*>(sA + (i21_base + t * i21_step) + off) = g_pack(vv.x, vv.y);
+                        cur = g_cmul(cur, twb);
+                      }
+                    });
       }
       // gate rows of this stage, loaded while the last level runs
       load_pairs(xptr[n], r0, r1, tb);
@@ -528,16 +615,15 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
     {
       __nv_bfloat16* y0 = y + r0 + tb;
       __nv_bfloat16* y1 = y + r1 + tb;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      g_pipe4<16>(i1_addr, [&](int i, const uint32_t (&r)[16]) {
         float2 zz[8];
-        z_row(i, false, zz);
+        z_of(i, r, false, 1.f, zz);
 #pragma unroll
         for (int n3 = 0; n3 < 8; ++n3) {
           y0[32 * i + 1024 * n3] = __float2bfloat16_rn(zz[n3].x);
           y1[32 * i + 1024 * n3] = __float2bfloat16_rn(zz[n3].y);
         }
-      }
+      });
     }
     // the next pair's first level overwrites TMEM: order these reads before it
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

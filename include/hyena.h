@@ -30,11 +30,11 @@
  *    (see hyena_last_cuda_error()).
  *  - Activations v, x_n, y are row-major [B][D][L] (time fastest) in the
  *    storage type `dtype`; bf16 results are rounded to nearest even. The
- *    arithmetic is float32, except that hyena_forward with bf16 I/O, B even
- *    and L in {1024, 2048, 8192} runs its transforms on the tensor cores with
- *    f16 operands (scaled by exact powers of two) and float32 accumulation;
- *    that adds an error below the bf16 output rounding (relative L2 within
- *    the bf16 tolerance of 8e-3).
+ *    arithmetic is float32, except that hyena_forward with bf16 I/O and B
+ *    even runs its transforms on the tensor cores with f16 operands (scaled
+ *    by exact powers of two) and float32 accumulation for L in {1024, 2048}
+ *    and, up to order N = 3, for L = 8192; that adds an error of the order of
+ *    the bf16 output rounding (relative L2 within the bf16 tolerance of 8e-3).
  *  - For the 1-D FFT calls L must be a power of two with 16 <= L <= 2^20
  *    (HYENA_ERR_UNSUPPORTED otherwise); 1 <= N <= 8; B, D >= 1. The
  *    StripedHyena calls take any L >= 1 and the HyenaND calls state their
@@ -342,7 +342,7 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
  * Kernels that wait on mbarriers for asynchronous copies or tensor-core
  * completions (the striped bulk-copy kernel of hyena_striped_forward, taken
  * when a row's byte length is a multiple of 16, and the tcgen05 forward of
- * hyena_forward for bf16, B even, L = 8192) bound every wait in time: a
+ * hyena_forward for bf16, B even, L = 8192, N <= 3) bound every wait in time: a
  * wait gives up 0.2 s of GPU global time after it started (each polling
  * step suspends for at most 20 us). A wait that runs out makes every thread
  * block of that launch stop early (its outputs are then invalid) and sets a

@@ -1,9 +1,10 @@
-"""The tcgen05 forward (bf16 I/O, B even, L = 8192): every DFT level of the
-2L-point pair transform is a GEMM on the tensor cores (f16 operands scaled by
-exact powers of two, float32 accumulation in TMEM).
+"""The tcgen05 forward (bf16 I/O, B even, L = 8192, order N <= 3): every DFT
+level of the 2L-point pair transform is a GEMM on the tensor cores (f16
+operands scaled by exact powers of two, float32 accumulation in TMEM).
 
 Checked through the binding (C ABI) against the float64 oracle on every row
-of small shapes (orders 1 to 8, even B; odd B runs the SIMT kernel), its
+of small shapes (orders 1 to 3 with even B; odd B and orders 4 to 8 run the
+float32 SIMT kernel, whose results are checked the same way), its
 spectrum copy against the oracle spectrum, its dispatch (one launch of the
 tcgen05 kernel per forward, read from a CUDA-graph capture), exact
 power-of-two scaling, and the cleared timeout flag. The full-size workload at
@@ -71,9 +72,10 @@ def _kernel_names(hy, w, tv, txs, hh):
     return names
 
 
-@pytest.mark.parametrize("B,expect", [(2, "tcg_forward_kernel"), (3, "fused_forward_kernel")])
-def test_dispatch(hy, B, expect):
-    w = synth.custom(2, "bf16", B, 2, L, seed=3)
+@pytest.mark.parametrize("N,B,expect", [(2, 2, "tcg_forward_kernel"), (3, 4, "tcg_forward_kernel"),
+                                         (2, 3, "fused_forward_kernel"), (4, 2, "fused_forward_kernel")])
+def test_dispatch(hy, N, B, expect):
+    w = synth.custom(N, "bf16", B, 2, L, seed=3)
     wt = synth.filter_weights(w)
     v, xs = synth.inputs(w)
     h = hy.filter_generate(weights_to_cuda(wt), w.N, w.D, w.L, w.alpha_lo, w.alpha_hi)
