@@ -202,7 +202,9 @@ hyena_status hyena_device_timeouts(void) {
   if (b < 0) return cuda_fail(cudaGetLastError());
   const int g = tcg_read_and_clear_timeout();
   if (g < 0) return cuda_fail(cudaGetLastError());
-  return (b || g) ? HYENA_ERR_TIMEOUT : HYENA_OK;
+  const int f = fourstep_read_and_clear_timeout();
+  if (f < 0) return cuda_fail(cudaGetLastError());
+  return (b || g || f) ? HYENA_ERR_TIMEOUT : HYENA_OK;
 }
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {

@@ -14,9 +14,22 @@
 // 2N + 1 launches per wave of channels; waves are sized by the workspace so
 // that the array stays resident in L2.
 #include "kernels.cuh"
+#include "mbar.cuh"
 #include "paired.cuh"
 
 namespace hyena {
+
+// Row pass spectrum rows fed by bulk copies into shared memory (issued when
+// the CTA starts, waited for before the paired pass) for rows of up to
+// 2^HYENA_ROW_BULK_MAX_LOG points, else read from global memory inside the
+// paired pass. Measured: rows of 1024 (L = 2^17) 0.702 -> 0.683 ms per
+// forward with the copies; rows of 4096 (L = 2^20) 7.69 -> 7.95 ms, where the
+// 64 KB of staged rows leave the one resident CTA less L1 for its scratch rows.
+#ifndef HYENA_ROW_BULK_MAX_LOG
+#define HYENA_ROW_BULK_MAX_LOG 10
+#endif
+
+__device__ int g_fourstep_timeout;
 
 enum ColMode { kColFirst = 0, kColMid = 1, kColLast = 2, kColSpecFirst = 3 };
 
@@ -133,6 +146,9 @@ col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict_
 
 // Row pass on rows kA and kB (kA + kB = M1, or the self-mirrored rows 0 and
 // M1/2 in CTA 0). Threads [0, TV) work on row kA, [TV, 2 TV) on row kB.
+// The two spectrum rows of the pair are fetched by one thread with two bulk
+// copies into shared memory while the forward row FFT runs (byte-counted on
+// an mbarrier, bounded wait before the paired pass).
 // Resident row-pair CTAs per SM the register budget is sized for: 512 threads
 // per SM (rows of 1024 points: 4 CTAs of 128 threads at <= 128 registers,
 // measured 8 % faster than the unbounded 137 registers and 3 CTAs).
@@ -141,13 +157,24 @@ constexpr int row_blocks() {
   return 512 / (2 * Plan<LOGMV>::TV) > 1 ? 512 / (2 * Plan<LOGMV>::TV) : 1;
 }
 
+template <int LOGMV, int MODE, typename HT>
+struct RowSmem {
+  static constexpr int MV = 1 << LOGMV;
+  static constexpr bool bulk = LOGMV <= HYENA_ROW_BULK_MAX_LOG && MODE == kPairConv;
+  static constexpr size_t data = sizeof(float2) * 2 * (size_t)padded_len(MV);
+  static constexpr size_t spec_row = sizeof(HT) * (size_t)MV;   // bytes of one staged spectrum row
+  static constexpr size_t total = data + (bulk ? 2 * spec_row : 0);
+};
+
 template <int LOGMV, int MODE, typename HT = float2>
 __global__ void __launch_bounds__(2 * Plan<LOGMV>::TV, row_blocks<LOGMV>())
 row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const float2* __restrict__ tables, int M1,
            int B, long long ch0) {
   using P = Plan<LOGMV>;
+  using RS = RowSmem<LOGMV, MODE, HT>;
   constexpr int MV = P::MV, TV = P::TV, Q8 = MV / 8, Q16 = MV / 16, VEC = padded_len(MV);
-  extern __shared__ float2 sm[];
+  extern __shared__ __align__(16) float2 sm[];
+  __shared__ __align__(8) uint64_t hbar;
   const int M = M1 * MV;
   const float2* __restrict__ tw = tables;
   const float2* __restrict__ Wv = tables + MV;
@@ -166,6 +193,18 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
   const int krow = vec ? kB : kA;
   float2* base = sm + vec * VEC;
   float2* src = S + (size_t)krow * MV;
+  HT* hs = reinterpret_cast<HT*>(reinterpret_cast<char*>(sm) + RS::data);   // staged rows kA, kB
+  if constexpr (RS::bulk) {
+    if (t == 0) {
+      const uint32_t bar = smem_u32(&hbar);
+      mbar_init(bar, 1);
+      mbar_init_fence();
+      mbar_arrive_expect_tx(bar, (uint32_t)(2 * RS::spec_row));
+      bulk_g2s(smem_u32(hs), H + (size_t)kA * MV, (uint32_t)RS::spec_row, bar);
+      bulk_g2s(smem_u32(hs + MV), H + (size_t)kB * MV, (uint32_t)RS::spec_row, bar);
+    }
+    // the barrier after the first forward pass publishes the initialised mbarrier
+  }
 
   // four-step twiddle w_M^{krow n2}, n2 = tl + r*Q16
   const float2 tw0 = expi_neg((int)(((long long)krow * tl) % M), M);
@@ -198,13 +237,14 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
       float s, c;
       sincospif((float)kA / (float)M, &s, &c);
       rho = make_float2(c, -s);
-      HA = H + (size_t)kA * MV; HB = H + (size_t)kB * MV;
+      HA = RS::bulk ? hs : H + (size_t)kA * MV;
+      HB = RS::bulk ? hs + MV : H + (size_t)kB * MV;
     } else if (t < Q16) {
       bA = bB = sm;
       head = (t == 0);
       jA = head ? 0 : t; jB = head ? Q16 : Q8 - t;
       rho = make_float2(1.f, 0.f); has_rho = false;
-      HA = HB = H;
+      HA = HB = RS::bulk ? hs : H;
     } else {
       const int t2 = t - Q16;
       bA = bB = sm + VEC;
@@ -212,9 +252,15 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
       float s, c;
       sincospif((float)(M1 / 2) / (float)M, &s, &c);
       rho = make_float2(c, -s);
-      HA = HB = H + (size_t)(M1 / 2) * MV;
+      HA = HB = RS::bulk ? hs + MV : H + (size_t)(M1 / 2) * MV;
     }
-    paired_pass<LOGMV, MODE, false, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
+    if constexpr (RS::bulk) {
+      if (!mbar_wait(smem_u32(&hbar), 0)) atomicExch(&g_fourstep_timeout, 1);
+      paired_pass<LOGMV, MODE, true, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
+    } else {
+      paired_pass<LOGMV, MODE, false, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB,
+                                          1.0f / (8.0f * (float)M));
+    }
   }
   if (MODE == kPairSpectrum) return;
   __syncthreads();
@@ -258,7 +304,7 @@ template <int LOGMV, int MODE, typename HT = float2>
 static cudaError_t launch_row(float2* scr, const float2* spec, const float2* tables, int M1, int B, long long ch0,
                               int nch, cudaStream_t s) {
   auto k = row_kernel<LOGMV, MODE, HT>;
-  const size_t smem = sizeof(float2) * 2 * (size_t)padded_len(1 << LOGMV);
+  const size_t smem = RowSmem<LOGMV, MODE, HT>::total;
   cudaError_t e = prep(k, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(M1 / 2, nch);
@@ -336,6 +382,16 @@ static cudaError_t spec_l(const float* h, float2* spec, const float2* tables, in
     case 16: return spec_lm<LOGMV, 16>(h, spec, tables, D, y, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+int fourstep_read_and_clear_timeout() {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fourstep_timeout, sizeof(int)) != cudaSuccess) return -1;
+  if (v) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fourstep_timeout, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
 }
 
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D, const Layout& y,

@@ -100,6 +100,7 @@ cudaError_t launch_striped(const void* xq, const void* xk, const void* xv, const
 int striped_read_and_clear_timeout();
 cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D, int L, float* h, cudaStream_t s);
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
+int fourstep_read_and_clear_timeout();
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
                                      const Layout& y, cudaStream_t s);
 cudaError_t launch_filter_generate(const float* W1, const float* b1, const float* W2, const float* b2,

@@ -14,6 +14,7 @@
 // pages' 1-based t - 1 is the 0-based lag t).
 #include "fft_engine.cuh"
 #include "kernels.cuh"
+#include "mbar.cuh"
 
 namespace hyena {
 
@@ -217,41 +218,6 @@ striped_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T* __re
 
 __device__ int g_striped_timeout;
 
-__device__ __forceinline__ uint32_t st_smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ unsigned long long st_globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for the phase of an mbarrier to complete, bounded in time: each
-// try_wait suspends for at most kStTrySuspendNs, and the wait gives up once
-// kStWaitLimitNs of global time have passed since it started (returns false).
-constexpr unsigned kStTrySuspendNs = 20000;                 // 20 us per try
-constexpr unsigned long long kStWaitLimitNs = 200000000ull; // 0.2 s per wait
-__device__ __forceinline__ bool st_mbar_wait(uint32_t bar, uint32_t phase,
-                                             unsigned long long limit_ns = kStWaitLimitNs) {
-  const unsigned long long t0 = st_globaltimer_ns();
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
-        "selp.b32 %0, 1, 0, P1;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(phase), "r"(kStTrySuspendNs)
-        : "memory");
-    if (done) return true;
-    if (st_globaltimer_ns() - t0 > limit_ns) return false;
-  }
-}
-
 template <typename T>
 __device__ __forceinline__ float ldsT(const T* p);
 template <>
@@ -349,8 +315,8 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
   const T* srcs[3] = {xq, xk, xv};
 
   if (tid == 0) {
-    for (int k = 0; k < 2; ++k) asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(st_smem_u32(&bars[k])), "r"(1));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int k = 0; k < 2; ++k) mbar_init(smem_u32(&bars[k]), 1);
+    mbar_init_fence();
   }
   __syncthreads();
 
@@ -361,10 +327,10 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
     const int n = min(kStTile, L - t0);
     const int h = t0 >= HP ? HP : 0;               // first tile: halo zero-filled by the threads
     const uint32_t bytes = (uint32_t)((h + n) * E);
-    const uint32_t bar = st_smem_u32(&bars[stage]);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(3 * bytes) : "memory");
+    const uint32_t bar = smem_u32(&bars[stage]);
+    mbar_arrive_expect_tx(bar, 3 * bytes);
     for (int a = 0; a < 3; ++a)
-      bulk_g2s(st_smem_u32(win(stage, a) + (HP - h)), srcs[a] + (size_t)rowi * L + t0 - h, bytes, bar);
+      bulk_g2s(smem_u32(win(stage, a) + (HP - h)), srcs[a] + (size_t)rowi * L + t0 - h, bytes, bar);
   };
 
   uint32_t phase[2] = {0, 0};
@@ -386,7 +352,7 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
       issue(it + gridDim.x, stage ^ 1);
       pending[stage ^ 1] = true;
     }
-    const bool done = st_mbar_wait(st_smem_u32(&bars[stage]), phase[stage]);
+    const bool done = mbar_wait(smem_u32(&bars[stage]), phase[stage]);
     if (done) {
       phase[stage] ^= 1;
       pending[stage] = false;
@@ -459,7 +425,7 @@ striped_bulk_kernel(const T* __restrict__ xq, const T* __restrict__ xk, const T*
   // into this CTA's shared memory before it exits (normal exits leave none)
   if (tid == 0)
     for (int k = 0; k < 2; ++k)
-      if (pending[k]) st_mbar_wait(st_smem_u32(&bars[k]), phase[k], 1000000000ull);
+      if (pending[k]) mbar_wait(smem_u32(&bars[k]), phase[k], 1000000000ull);
   __syncthreads();
 }
 

@@ -39,6 +39,7 @@
 
 #include "fft_engine.cuh"
 #include "kernels.cuh"
+#include "mbar.cuh"
 
 namespace hyena {
 
@@ -76,7 +77,6 @@ __host__ __device__ constexpr uint32_t g_idesc(int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-__device__ __forceinline__ uint32_t g_smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
 __device__ __forceinline__ uint64_t g_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
@@ -92,38 +92,6 @@ __device__ __forceinline__ void g_mma(uint32_t dtmem, uint64_t da, uint64_t db, 
 
 __device__ __forceinline__ void g_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, multiple of 16 bytes).
-__device__ __forceinline__ void g_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ unsigned long long g_globaltimer_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for an mbarrier phase, bounded in time (each try suspends for at most
-// HYENA_TCG_SUSPEND_NS; false once limit_ns of global time have passed).
-constexpr unsigned long long kGWaitLimitNs = 200000000ull;   // 0.2 s
-#ifndef HYENA_TCG_SUSPEND_NS
-#define HYENA_TCG_SUSPEND_NS 20000
-#endif
-__device__ __forceinline__ bool g_wait(uint32_t bar, uint32_t phase, unsigned long long limit_ns = kGWaitLimitNs) {
-  const unsigned long long t0 = g_globaltimer_ns();
-  for (;;) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2, %3;\n\t"
-        "selp.b32 %0, 1, 0, P1;\n\t}\n"
-        : "=r"(done)
-        : "r"(bar), "r"(phase), "r"((uint32_t)HYENA_TCG_SUSPEND_NS)
-        : "memory");
-    if (done) return true;
-    if (g_globaltimer_ns() - t0 > limit_ns) return false;
-  }
 }
 
 #define G_LD_REGS16(r, o)                                                                                      \
@@ -268,10 +236,10 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
   float* red = reinterpret_cast<float*>(sm + kOffMisc + 16);
   const __nv_bfloat16** xptr = reinterpret_cast<const __nv_bfloat16**>(sm + kOffPtr);
   const unsigned char** hptr = reinterpret_cast<const unsigned char**>(sm + kOffPtr + 8 * kMaxOrder);
-  const uint32_t aA = g_smem_u32(sA), aB = g_smem_u32(sB), abar = g_smem_u32(bar);
+  const uint32_t aA = smem_u32(sA), aB = smem_u32(sB), abar = smem_u32(bar);
 
   if (w == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(g_smem_u32(tslot)),
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
                  "r"(kGCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
   }
@@ -280,8 +248,8 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
     hptr[tid] = reinterpret_cast<const unsigned char*>(hh.p[tid]);
   }
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(abar), "r"(1));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init(abar, 1);
+    mbar_init_fence();
   }
   g_build_dft(sB, kBF1, 16, 16, 8, false, 0x1p-4f, tid);
   g_build_dft(sB, kBF32, 32, 32, 32, false, 0x1p-8f, tid);
@@ -335,7 +303,7 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
       issue();
       g_commit(abar);
     }
-    ok = g_wait(abar, phase);
+    ok = mbar_wait(abar, phase);
     phase ^= 1;
     if (!ok) atomicExch(&g_tcg_timeout, 1);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -413,14 +381,14 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
       // reads from HBM later: its spectrum row, its gate rows, and after the
       // last stage the next pair's input rows
       if (tid == 0) {
-        g_prefetch_l2(hrow, (uint32_t)kGHRowBytes);
-        g_prefetch_l2(xptr[n] + r0, 2 * kGL);
-        g_prefetch_l2(xptr[n] + r1, 2 * kGL);
+        bulk_prefetch_l2(hrow, (uint32_t)kGHRowBytes);
+        bulk_prefetch_l2(xptr[n] + r0, 2 * kGL);
+        bulk_prefetch_l2(xptr[n] + r1, 2 * kGL);
         if (n + 1 == N && p + gridDim.x < npairs) {
           const long long pn = p + gridDim.x;
           const size_t q0 = ((size_t)(2 * (int)(pn % Bh)) * D + (size_t)(pn / Bh)) * (size_t)kGL;
-          g_prefetch_l2(v + q0, 2 * kGL);
-          g_prefetch_l2(v + q0 + (size_t)D * kGL, 2 * kGL);
+          bulk_prefetch_l2(v + q0, 2 * kGL);
+          bulk_prefetch_l2(v + q0 + (size_t)D * kGL, 2 * kGL);
         }
       }
       const bool first = (n == 0);
@@ -630,7 +598,7 @@ tcg_forward_kernel(const __nv_bfloat16* __restrict__ v, GatePtrs<__nv_bfloat16> 
   }
 done:
   // after a timeout: wait (bounded, 1 s) for the MMAs of the last issued level
-  if (!ok) g_wait(abar, phase ^ 1, 1000000000ull);
+  if (!ok) mbar_wait(abar, phase ^ 1, 1000000000ull);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kGCols));
