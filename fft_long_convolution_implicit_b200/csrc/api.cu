@@ -109,11 +109,20 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
   } else {
     const size_t per = sizeof(float2) * (size_t)ly.M;
     const long long C = (long long)B * D;
-    long long w = (long long)(workspace_bytes / per);
+    // tensor-core rows when the workspace also holds the per-channel maxima
+    bool tcr = allow_tc && bf16 && !spec16 && N <= kTcgMaxOrder && tcr_layout(ly) &&
+               workspace_bytes >= per + kTcrChannelExtraBytes;
+    long long w = (long long)(workspace_bytes / (tcr ? per + kTcrChannelExtraBytes : per));
     if (w < 1) return cudaErrorInvalidValue;
     if (w > C) w = C;
     if (w > kMaxGridY) w = kMaxGridY;
     FourStepLaunch p{};
+    p.tcr = tcr;
+    if (tcr) {
+      p.xmax = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(workspace) + per * (size_t)w);
+      for (int n = 0; n < N; ++n)
+        p.hmax[n] = reinterpret_cast<const float*>(reinterpret_cast<const float2*>(hhat[n]) + hmax_offset(ly, D));
+    }
     p.v = v;
     for (int n = 0; n < N; ++n) {
       p.x[n] = x[n];
@@ -128,7 +137,8 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     for (long long c0 = 0; c0 < C && e == cudaSuccess; c0 += w) {
       p.ch0 = c0;
       p.wave = (int)((C - c0) < w ? (C - c0) : w);
-      e = launch_fourstep_wave(p, ly, s);
+      if (tcr) e = cudaMemsetAsync(p.xmax, 0, sizeof(unsigned) * 2 * (size_t)p.wave, s);
+      if (e == cudaSuccess) e = launch_fourstep_wave(p, ly, s);
     }
   }
   return e;
@@ -156,7 +166,7 @@ size_t hyena::fourstep_wave_bytes(long long channels, const Layout& ly) {
   if (w < 1) w = 1;
   if (w > channels) w = channels;
   if (w > kMaxGridY) w = kMaxGridY;
-  return per * (size_t)w;
+  return (per + (tcr_layout(ly) ? kTcrChannelExtraBytes : 0)) * (size_t)w;
 }
 
 cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, const Layout& ly, bool with_tc,
@@ -175,6 +185,8 @@ cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, con
       const int nd = (int)((rows - c0) < kMaxGridY ? (rows - c0) : kMaxGridY);
       e = launch_fourstep_spectrum(h + (size_t)c0 * ly.L, spec + (size_t)c0 * ly.M, tables, nd, ly, s);
     }
+    if (e == cudaSuccess && tcr_layout(ly))
+      e = launch_tcr_hmax(spec, rows, ly.M, reinterpret_cast<float*>(spec + hmax_offset(ly, rows)), s);
   }
   return e;
 }
@@ -204,7 +216,9 @@ hyena_status hyena_device_timeouts(void) {
   if (g < 0) return cuda_fail(cudaGetLastError());
   const int f = fourstep_read_and_clear_timeout();
   if (f < 0) return cuda_fail(cudaGetLastError());
-  return (b || g || f) ? HYENA_ERR_TIMEOUT : HYENA_OK;
+  const int r = tcr_read_and_clear_timeout();
+  if (r < 0) return cuda_fail(cudaGetLastError());
+  return (b || g || f || r) ? HYENA_ERR_TIMEOUT : HYENA_OK;
 }
 
 hyena_status hyena_spectrum_layout(int L, int* M, int* M1, int* MV) {

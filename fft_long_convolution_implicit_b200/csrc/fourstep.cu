@@ -59,7 +59,7 @@ template <int MB, int MODE, typename T>
 __global__ void __launch_bounds__(ColCfg<MB>::THREADS)
 col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict__ yout, float2* __restrict__ scr,
            const float2* __restrict__ tw1, int B, int D, int L, int MV, long long ch0,
-           const float* __restrict__ inv_scale) {
+           const float* __restrict__ inv_scale, unsigned* __restrict__ xmax) {
   using Cfg = ColCfg<MB>;
   constexpr int M1 = Cfg::M1, CW = Cfg::CW, NQ = 16 / MB;
   extern __shared__ float2 sm[];
@@ -121,9 +121,20 @@ col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict_
   }
   // forward column transform (upper half of the column is zero)
   dft16<false, true, false, 0>(a);
+  // largest component of the channel's column outputs (float bits order as
+  // unsigned integers for non-negative values), for the tensor-core row pass
+  auto record_max = [&]() {
+    if (xmax == nullptr) return;
+    float mx = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) mx = fmaxf(mx, fmaxf(fabsf(a[r].x), fabsf(a[r].y)));
+    const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+    if ((threadIdx.x & 31) == 0) atomicMax(xmax + blockIdx.y, m);
+  };
   if constexpr (MB == 1) {
 #pragma unroll
     for (int r = 0; r < 16; ++r) S[(size_t)r * MV + n2] = a[r];
+    record_max();
   } else {
 #pragma unroll
     for (int r = 0; r < 16; ++r) csm[pidx(16 * j + r)] = a[r];
@@ -141,6 +152,7 @@ col_kernel(const T* __restrict__ zin, const T* __restrict__ gate, T* __restrict_
     for (int q = 0; q < NQ; ++q)
 #pragma unroll
       for (int r = 0; r < MB; ++r) S[(size_t)(j + q * MB + 16 * r) * MV + n2] = a[q * MB + r];
+    record_max();
   }
 }
 
@@ -290,13 +302,13 @@ static cudaError_t prep(K kernel, size_t smem) {
 template <int MB, int MODE, typename T>
 static cudaError_t launch_col(const T* zin, const T* gate, T* yout, float2* scr, const float2* tw1, int B, int D,
                               int L, int MV, long long ch0, int nch, cudaStream_t s,
-                              const float* inv_scale = nullptr) {
+                              const float* inv_scale = nullptr, unsigned* xmax = nullptr) {
   using Cfg = ColCfg<MB>;
   auto k = col_kernel<MB, MODE, T>;
   cudaError_t e = prep(k, Cfg::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid(MV / Cfg::CW, nch);
-  k<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(zin, gate, yout, scr, tw1, B, D, L, MV, ch0, inv_scale);
+  k<<<grid, Cfg::THREADS, Cfg::SMEM, s>>>(zin, gate, yout, scr, tw1, B, D, L, MV, ch0, inv_scale, xmax);
   return cudaGetLastError();
 }
 
@@ -316,17 +328,25 @@ template <int LOGMV, int MB, typename T, typename HT>
 static cudaError_t wave_t(const FourStepLaunch& p, const Layout& y, cudaStream_t s) {
   const float2* tw1 = p.tables + y.tw_1;
   const int MV = y.MV;
+  // tensor-core rows: stage n reads the column maxima in buffer n & 1 and
+  // clears the other for the column pass that feeds stage n + 1
+  unsigned* xm[2] = {p.tcr ? p.xmax : nullptr, p.tcr ? p.xmax + p.wave : nullptr};
   cudaError_t e = launch_col<MB, kColFirst, T>(reinterpret_cast<const T*>(p.v), nullptr, nullptr, p.scratch, tw1,
-                                               p.B, p.D, p.L, MV, p.ch0, p.wave, s);
+                                               p.B, p.D, p.L, MV, p.ch0, p.wave, s, nullptr, xm[0]);
   for (int n = 0; n < p.N && e == cudaSuccess; ++n) {
-    e = launch_row<LOGMV, kPairConv, HT>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);
+    if (p.tcr)
+      e = launch_tcr_rows(p.scratch, p.hh.p[n], p.hmax[n], xm[n & 1], xm[(n + 1) & 1], y.M1, p.B, p.ch0, p.wave,
+                          s);
+    else
+      e = launch_row<LOGMV, kPairConv, HT>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);
     if (e != cudaSuccess) break;
     const float* inv = nullptr;
     if (sizeof(HT) != sizeof(float2))
       inv = reinterpret_cast<const float*>(reinterpret_cast<const char*>(p.hh.p[n]) + spec16_scales_offset_bytes(y, p.D));
     const T* g = reinterpret_cast<const T*>(p.x[n]);
     if (n + 1 < p.N)
-      e = launch_col<MB, kColMid, T>(nullptr, g, nullptr, p.scratch, tw1, p.B, p.D, p.L, MV, p.ch0, p.wave, s, inv);
+      e = launch_col<MB, kColMid, T>(nullptr, g, nullptr, p.scratch, tw1, p.B, p.D, p.L, MV, p.ch0, p.wave, s, inv,
+                                     xm[(n + 1) & 1]);
     else
       e = launch_col<MB, kColLast, T>(nullptr, g, reinterpret_cast<T*>(p.y), p.scratch, tw1, p.B, p.D, p.L, MV,
                                       p.ch0, p.wave, s, inv);

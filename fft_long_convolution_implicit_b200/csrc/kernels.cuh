@@ -55,6 +55,11 @@ struct FourStepLaunch {
   long long ch0;     // first channel (c-major order) of this wave
   int wave;          // channels in this wave
   bool spec16;       // spectrum blocks in the reduced-precision (__half2) format
+  // tensor-core row pass (rows of 4096, bf16, order <= kTcgMaxOrder): two
+  // buffers of `wave` per-channel maxima (float bits) of the column pass output
+  bool tcr;
+  unsigned* xmax;
+  const float* hmax[kMaxOrder];   // per filter: the spectrum block's per-channel maxima
 };
 
 // Records e as this thread's last CUDA error (hyena_last_cuda_error) and
@@ -101,6 +106,11 @@ int striped_read_and_clear_timeout();
 cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D, int L, float* h, cudaStream_t s);
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
 int fourstep_read_and_clear_timeout();
+// tensor-core row pass of one four-step stage (rows of 4096 points)
+cudaError_t launch_tcr_rows(float2* scr, const float2* spec, const float* hmax, const unsigned* xmax,
+                            unsigned* xmax_clear, int M1, int B, long long ch0, int wave, cudaStream_t s);
+cudaError_t launch_tcr_hmax(const float2* spec, int D, int M, float* hmax, cudaStream_t s);
+int tcr_read_and_clear_timeout();
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
                                      const Layout& y, cudaStream_t s);
 cudaError_t launch_filter_generate(const float* W1, const float* b1, const float* W2, const float* b2,

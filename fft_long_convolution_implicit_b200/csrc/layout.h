@@ -103,7 +103,16 @@ inline size_t tc_spectrum_offset(const Layout& y, int D) { return (size_t)D * y.
 inline size_t tables_offset(const Layout& y, int D) {
   return (size_t)D * y.M + (has_tc_copy(y) ? (size_t)D * tc_row(y) : 0);
 }
-inline size_t spectrum_block_floats2(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
+// Four-step layouts with rows of 4096 points may run their row pass on the
+// tensor cores; their spectrum block ends with each channel's largest
+// spectrum component ([D] float, padded to float2), and their workspace holds
+// two words per channel beside the scratch (the column pass's per-channel maxima).
+inline bool tcr_layout(const Layout& y) { return y.fourstep && y.logMV == 12; }
+inline size_t hmax_offset(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
+inline size_t spectrum_block_floats2(const Layout& y, int D) {
+  return hmax_offset(y, D) + (tcr_layout(y) ? (size_t)(D + 1) / 2 : 0);
+}
+constexpr size_t kTcrChannelExtraBytes = 8;
 
 // Reduced-precision spectrum block: [D][M] __half2 bins (same order, each
 // channel scaled by a power of two), [D] float 1 / scale (padded to 16 bytes),

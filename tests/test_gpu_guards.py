@@ -95,6 +95,7 @@ def run_guarded(hy, w, fill, f16=False):
     (2, "f32", 2, 2, 16384, False),      # fused SIMT, 1024 threads per channel
     (2, "bf16", 1, 3, 32768, False),     # four-step
     (2, "bf16", 1, 5, 131072, False),    # four-step, rows of 1024
+    (2, "bf16", 1, 3, 524288, False),    # four-step, rows of 4096 on the tensor cores
     (2, "bf16", 2, 2, 8192, True),       # f16 spectra, fused
     (2, "bf16", 1, 2, 65536, True),      # f16 spectra, four-step
 ])
