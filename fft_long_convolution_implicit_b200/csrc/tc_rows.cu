@@ -368,20 +368,22 @@ done:
   if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kRCols));
 }
 
-// Largest component of each channel's spectrum block rows (one CTA per channel).
-__global__ void tcr_hmax_kernel(const float2* __restrict__ spec, int M, float* __restrict__ hmax) {
-  __shared__ float red[8];
-  const float2* r = spec + (size_t)blockIdx.x * M;
+// Largest component of each channel's spectrum block rows: kHmaxSplit CTAs
+// per channel, 16-byte loads, the maximum merged as float bits (non-negative
+// floats order as unsigned integers) into hmax, which starts at zero.
+constexpr int kHmaxSplit = 16;
+__global__ void tcr_hmax_kernel(const float2* __restrict__ spec, int M, unsigned* __restrict__ hmax) {
+  const int c = blockIdx.x / kHmaxSplit, part = blockIdx.x % kHmaxSplit;
+  const int n4 = M / 2 / kHmaxSplit;   // float4 (two bins) per CTA
+  const float4* r = reinterpret_cast<const float4*>(spec + (size_t)c * M) + (size_t)part * n4;
   float mx = 0.f;
-  for (int i = threadIdx.x; i < M; i += blockDim.x) mx = fmaxf(mx, fmaxf(fabsf(r[i].x), fabsf(r[i].y)));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int k = 1; k < (int)(blockDim.x >> 5); ++k) mx = fmaxf(mx, red[k]);
-    hmax[blockIdx.x] = fmaxf(mx, red[0]);
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = __ldcs(r + i);
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
   }
+  const unsigned m = __reduce_max_sync(0xffffffffu, __float_as_uint(mx));
+  if ((threadIdx.x & 31) == 0) atomicMax(hmax + c, m);
 }
 
 cudaError_t launch_tcr_rows(float2* scr, const float2* spec, const float* hmax, const unsigned* xmax,
@@ -403,7 +405,9 @@ cudaError_t launch_tcr_rows(float2* scr, const float2* spec, const float* hmax, 
 }
 
 cudaError_t launch_tcr_hmax(const float2* spec, int D, int M, float* hmax, cudaStream_t s) {
-  tcr_hmax_kernel<<<D, 256, 0, s>>>(spec, M, hmax);
+  cudaError_t e = cudaMemsetAsync(hmax, 0, sizeof(float) * (size_t)D, s);
+  if (e != cudaSuccess) return e;
+  tcr_hmax_kernel<<<D * kHmaxSplit, 256, 0, s>>>(spec, M, reinterpret_cast<unsigned*>(hmax));
   return cudaGetLastError();
 }
 

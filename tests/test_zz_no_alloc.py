@@ -9,9 +9,11 @@ must not leak into the next result): the results are bit for bit equal (the
 two calls differ only in how many channels a wave holds, and every channel's
 arithmetic is the same whatever the wave), one row is checked against the
 float64 oracle, and the device's free memory is the same before and after a
-call (nothing is allocated). The shapes include L = 2^20, where the 16 MiB
-scratch holds two channels per wave and the last wave is partial. This file
-is collected last.
+call (nothing is allocated). The shapes include L = 2^20: in float32 the
+16 MiB scratch holds two channels per wave and the last wave is partial; in
+bf16 (order <= 3) the row pass runs on the tensor cores and also keeps the
+column pass's per-channel maxima in the scratch, so a wave holds one channel.
+This file is collected last.
 """
 import ctypes
 
@@ -25,7 +27,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("N,dtype,B,D,L", [(2, "bf16", 2, 3, 32768), (2, "bf16", 1, 40, 131072),
-                                           (3, "f32", 1, 2, 32768), (2, "bf16", 1, 3, 1 << 20)])
+                                           (3, "f32", 1, 2, 32768), (2, "bf16", 1, 3, 1 << 20),
+                                           (2, "f32", 1, 3, 1 << 20)])
 def test_static_workspace_matches_workspace_forward(N, dtype, B, D, L):
     import torch
     from fft_long_convolution_implicit_b200 import build
