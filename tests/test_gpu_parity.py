@@ -41,6 +41,26 @@ def test_filter_generate_matches_oracle(hy, cfg_i):
     assert err.max() < 1e-6, err.max()
 
 
+@pytest.mark.parametrize("width,n_bands,L,N,D", [(64, 8, 16, 1, 3), (64, 8, 4096, 3, 200), (64, 3, 32, 2, 130),
+                                                  (48, 5, 1024, 2, 3)])
+def test_filter_generate_shapes(hy, width, n_bands, L, N, D):
+    """Tap tails shorter than a tile, output counts that are not a multiple of
+    the last layer's block, other band counts, and a width other than 64
+    (served by the general kernel), against the float64 oracle on every row.
+    Bar: float32 evaluation of the same sums (either summation order, emulated
+    in numpy) reaches 1.8e-6 per-row relative L2 on the 600-row shape, on rows
+    where the 64-term last layer cancels; every row must stay within 5e-6 and
+    the mean within 1e-6."""
+    import dataclasses
+    w = dataclasses.replace(synth.custom(N, "f32", 1, D, L, seed=31 + L + D), width=width, n_bands=n_bands)
+    wt = synth.filter_weights(w)
+    h = hy.filter_generate(weights_to_cuda(wt), N, D, L, w.alpha_lo, w.alpha_hi, n_bands=n_bands)
+    got = h.cpu().numpy().reshape(N * D, L)
+    ref = oracle.implicit_filter(wt, N, D, L, w.alpha_lo, w.alpha_hi, n_bands=n_bands)
+    err = rel_l2_rows(got, ref)
+    assert err.max() < 5e-6 and err.mean() < 1e-6, (err.max(), err.mean())
+
+
 # -------------------------------------------------------------- spectrum ---
 
 @pytest.mark.parametrize("L", [16, 128, 1024, 2048, 8192, 16384, 65536, 131072])
