@@ -73,7 +73,8 @@ L2_BYTES = 126 * 2 ** 20
 # sources the dominant kernel of each path is compiled from
 KERNEL_FILES = {
     "fused": ("fused.cu", "fft_engine.cuh", "paired.cuh", "layout.h"),
-    "fourstep": ("fourstep.cu", "tc_rows.cu", "tcgen05.cuh", "mbar.cuh", "fft_engine.cuh", "paired.cuh", "layout.h"),
+    "fourstep": ("fourstep.cu", "tc_rows.cu", "tcgen05.cuh", "mbar.cuh", "fft_engine.cuh", "paired.cuh", "layout.h",
+                 "api.cu"),   # api.cu sizes the waves, which set the DRAM traffic
     "tc": ("tc_fused.cu", "tc_dft.cuh", "fft_engine.cuh", "layout.h"),
     "tcg": ("tc_gemm.cu", "tcgen05.cuh", "mbar.cuh", "fft_engine.cuh", "layout.h"),
 }

@@ -21,10 +21,21 @@ hyena_status cuda_fail(cudaError_t e) {
 
 bool aligned16(const void* p) { return p && ((reinterpret_cast<uintptr_t>(p) & 15u) == 0); }
 
-// Four-step channels run in waves whose scratch stays resident in L2: a wave
-// takes 3/4 of the device's L2 capacity (measured against 1/4 and 3/8 at
-// L = 2^20: 7.94 ms against 8.92 and 8.31 ms per forward; within 1.5 % at L = 2^17).
+// Four-step channels run in waves through the workspace. The workspace size
+// hyena_forward_workspace_bytes asks for depends on the row kernel:
+// - rows of 4096 on the tensor cores: a wave whose scratch stays resident in
+//   L2 between its passes, 5/8 of the device's L2 (order 2, bf16, D = 256:
+//   6.27 / 3.04 ms per forward at L = 2^20 / 2^19 against 6.73 / 3.26 ms at
+//   3/4 of L2; at these sizes the wave also cuts DRAM traffic from 89 to
+//   56 MB per channel at L = 2^20);
+// - the SIMT row kernels, bound by latency rather than DRAM: one wave of up
+//   to kWaveMaxBytes, i.e. fewer launches and fewer partly filled last rounds
+//   (L = 2^17, bf16: 0.601 against 0.665 ms per forward at 3/4 of L2; L = 2^20,
+//   f32: 6.97 against 7.71 ms);
+// - the backward's forward transforms: 3/4 of the L2 (as measured for it).
 constexpr size_t kWaveL2Num = 6, kWaveL2Den = 8;
+constexpr size_t kWaveTcrL2Num = 5, kWaveTcrL2Den = 8;
+constexpr size_t kWaveMaxBytes = size_t(1) << 30;
 constexpr size_t kWaveFallbackL2 = size_t(126) << 20;
 constexpr long long kMaxGridY = 65535;
 
@@ -160,9 +171,12 @@ static size_t device_l2_bytes() {
   return v;
 }
 
-size_t hyena::fourstep_wave_bytes(long long channels, const Layout& ly) {
+size_t hyena::fourstep_wave_bytes(long long channels, const Layout& ly, WaveRule rule) {
   const size_t per = sizeof(float2) * (size_t)ly.M;
-  long long w = (long long)(device_l2_bytes() * kWaveL2Num / kWaveL2Den / per);
+  const size_t budget = rule == WaveRule::kTensorRows ? device_l2_bytes() * kWaveTcrL2Num / kWaveTcrL2Den
+                        : rule == WaveRule::kSimtRows ? kWaveMaxBytes
+                                                      : device_l2_bytes() * kWaveL2Num / kWaveL2Den;
+  long long w = (long long)(budget / (per + (tcr_layout(ly) ? kTcrChannelExtraBytes : 0)));
   if (w < 1) w = 1;
   if (w > channels) w = channels;
   if (w > kMaxGridY) w = kMaxGridY;
@@ -263,7 +277,8 @@ size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dty
   if (B < 1 || D < 1 || N < 1 || N > kMaxOrder || (dtype != HYENA_F32 && dtype != HYENA_BF16)) return 0;
   if (!make_layout(L, &y)) return 0;
   if (!y.fourstep) return 0;
-  return fourstep_wave_bytes((long long)B * D, y);
+  const bool tensor_rows = dtype == HYENA_BF16 && N <= kTcgMaxOrder && tcr_layout(y);
+  return fourstep_wave_bytes((long long)B * D, y, tensor_rows ? WaveRule::kTensorRows : WaveRule::kSimtRows);
 }
 
 hyena_status hyena_forward(const void* v, const void* const* x, const void* const* hhat, int B, int D, int L,

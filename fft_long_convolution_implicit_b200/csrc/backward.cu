@@ -143,7 +143,7 @@ bool plan_backward(int B, int D, int N, const Layout& ly, BwdPlan* p) {
   if ((long long)2 * B * D > (1LL << 31) - 1) return false;
   p->SPEC2 = take(sizeof(float2) * spectrum_block_floats2(ly, 2 * B * D));
   p->SBLK = take(sizeof(float2) * spectrum_block_floats2(ly, D));
-  p->fws_bytes = ly.fourstep ? fourstep_wave_bytes((long long)B * D, ly) : 0;
+  p->fws_bytes = ly.fourstep ? fourstep_wave_bytes((long long)B * D, ly, WaveRule::kBackward) : 0;
   p->FWS = take(p->fws_bytes);
   p->total = o;
   return true;

@@ -75,7 +75,10 @@ cudaError_t forward_dispatch(const void* v, const void* const* x, const void* co
 // float32 spectrum block -> reduced-precision block (bins and scales; tables copied)
 cudaError_t launch_spectrum_to_f16(const float2* spec, unsigned char* out, int D, const Layout& y, cudaStream_t s);
 // Workspace of one L2-sized four-step wave over `channels` channels.
-size_t fourstep_wave_bytes(long long channels, const Layout& ly);
+// Workspace bytes for one wave of four-step channels (at most `channels`),
+// by the rule of the row kernel that will run (api.cu gives the measurements).
+enum class WaveRule { kTensorRows, kSimtRows, kBackward };
+size_t fourstep_wave_bytes(long long channels, const Layout& ly, WaveRule rule);
 // Spectrum block (spectra, optional tensor-core copy, tables) of `rows` real
 // rows h [rows][L] float32.
 cudaError_t spectrum_dispatch(const float* h, float2* spec, int rows, const Layout& ly, bool with_tc,

@@ -124,9 +124,12 @@ hyena_status hyena_spectrum_layout(int L, int *M, int *M1, int *MV);
 /*
  * Workspace bytes hyena_forward wants for this shape: 0 for L <= 16384 (the
  * fused kernel keeps everything on chip); for longer L, 8*L bytes per
- * channel for a wave of channels sized to stay resident in L2 (3/4 of the
- * current device's L2 capacity). Any workspace of at least 8*L bytes works
- * (smaller waves); 0 when the shape is invalid.
+ * channel (8*L + 8 when L is 2^19 or 2^20) for a wave of channels: sized to
+ * stay resident in L2 (5/8 of the current device's L2 capacity) where the
+ * row pass runs on the tensor cores (bf16, N <= 3, L = 2^19 or 2^20), else
+ * all channels up to 1 GiB (the SIMT row kernels are faster in fewer, larger
+ * waves). Any workspace of at least one channel's bytes works (smaller
+ * waves); 0 when the shape is invalid.
  */
 size_t hyena_forward_workspace_bytes(int B, int D, int L, int N, hyena_dtype dtype);
 

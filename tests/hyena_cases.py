@@ -66,16 +66,20 @@ def rel_l2_rows(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
     return np.where(den > 0, num / np.where(den > 0, den, 1), num)
 
 
-def wave_rows(w: synth.Workload, wave_channels: int, seed: int = 0) -> list[int]:
+def wave_rows(w: synth.Workload, wave_channels: int, seed: int = 0, min_rows: int = 8) -> list[int]:
     """Rows (b*D + c) that put at least one checked row in every wave of the
     four-step path: channels are taken in waves of `wave_channels` in
-    c-major order (channel index c*B + b); one row is drawn (seeded) from
-    every wave, and the first and last rows are always included."""
+    c-major order (channel index c*B + b); rows are drawn (seeded) from every
+    wave, enough per wave that at least `min_rows` are drawn in all, and the
+    first and last rows are always included."""
     rng = np.random.default_rng(1234 + seed)
     C = w.channels
+    waves = -(-C // wave_channels)
+    per_wave = max(1, -(-min_rows // waves))
     picks = {0, C - 1}
     for start in range(0, C, wave_channels):
-        ch = int(rng.integers(start, min(C, start + wave_channels)))
-        c, b = divmod(ch, w.B)
-        picks.add(b * w.D + c)
+        stop = min(C, start + wave_channels)
+        for ch in rng.choice(np.arange(start, stop), size=min(per_wave, stop - start), replace=False):
+            c, b = divmod(int(ch), w.B)
+            picks.add(b * w.D + c)
     return sorted(picks)

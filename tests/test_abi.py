@@ -53,6 +53,16 @@ def test_host_queries(lib):
     assert hy.forward_workspace_bytes(4, 768, 2048, 2, True) == 0
     ws = hy.forward_workspace_bytes(1, 256, 131072, 2, True)
     assert ws % (131072 * 8) == 0 and ws >= 131072 * 8
+    # SIMT rows: all channels in one wave, up to 1 GiB
+    assert ws == 256 * 131072 * 8
+    assert hy.forward_workspace_bytes(8, 256, 131072, 2, True) == 1024 * 131072 * 8
+    # tensor-core rows of 4096 (bf16, order <= 3): 5/8 of the L2, 8 more bytes per channel
+    per = 8 * (1 << 20) + 8
+    ws_t = hy.forward_workspace_bytes(1, 256, 1 << 20, 2, True)
+    assert ws_t % per == 0 and 1 <= ws_t // per <= 20
+    ws_s = hy.forward_workspace_bytes(1, 256, 1 << 20, 2, False)   # float32 I/O: SIMT rows
+    assert ws_s % per == 0 and ws_s // per == (1 << 30) // per
+    assert hy.forward_workspace_bytes(1, 256, 1 << 20, 4, True) == ws_s   # order 4: SIMT rows
     assert hy.forward_workspace_bytes(1, 1, 1000, 2, True) == 0       # unsupported L
     assert hy.filter_spectrum_bytes(4, 3000) == 0
 
