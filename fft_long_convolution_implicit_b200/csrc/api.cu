@@ -131,8 +131,10 @@ cudaError_t hyena::forward_dispatch(const void* v, const void* const* x, const v
     p.tcr = tcr;
     if (tcr) {
       p.xmax = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(workspace) + per * (size_t)w);
-      for (int n = 0; n < N; ++n)
+      for (int n = 0; n < N; ++n) {
         p.hmax[n] = reinterpret_cast<const float*>(reinterpret_cast<const float2*>(hhat[n]) + hmax_offset(ly, D));
+        p.hhalf[n] = reinterpret_cast<const uint32_t*>(reinterpret_cast<const float2*>(hhat[n]) + tcr_half_offset(ly, D));
+      }
     }
     p.v = v;
     for (int n = 0; n < N; ++n) {
@@ -201,6 +203,9 @@ cudaError_t hyena::spectrum_dispatch(const float* h, float2* spec, int rows, con
     }
     if (e == cudaSuccess && tcr_layout(ly))
       e = launch_tcr_hmax(spec, rows, ly.M, reinterpret_cast<float*>(spec + hmax_offset(ly, rows)), s);
+    if (e == cudaSuccess && with_tc && tcr_layout(ly))
+      e = launch_tcr_half(spec, reinterpret_cast<const float*>(spec + hmax_offset(ly, rows)), rows, ly.M,
+                          reinterpret_cast<uint32_t*>(spec + tcr_half_offset(ly, rows)), s);
   }
   return e;
 }

@@ -212,8 +212,9 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
       mbar_init(bar, 1);
       mbar_init_fence();
       mbar_arrive_expect_tx(bar, (uint32_t)(2 * RS::spec_row));
-      bulk_g2s(smem_u32(hs), H + (size_t)kA * MV, (uint32_t)RS::spec_row, bar);
-      bulk_g2s(smem_u32(hs + MV), H + (size_t)kB * MV, (uint32_t)RS::spec_row, bar);
+      const uint64_t pol = l2_policy_evict_first();   // spectrum rows are read once per stage
+      bulk_g2s_policy(smem_u32(hs), H + (size_t)kA * MV, (uint32_t)RS::spec_row, bar, pol);
+      bulk_g2s_policy(smem_u32(hs + MV), H + (size_t)kB * MV, (uint32_t)RS::spec_row, bar, pol);
     }
     // the barrier after the first forward pass publishes the initialised mbarrier
   }
@@ -335,7 +336,7 @@ static cudaError_t wave_t(const FourStepLaunch& p, const Layout& y, cudaStream_t
                                                p.B, p.D, p.L, MV, p.ch0, p.wave, s, nullptr, xm[0]);
   for (int n = 0; n < p.N && e == cudaSuccess; ++n) {
     if (p.tcr)
-      e = launch_tcr_rows(p.scratch, p.hh.p[n], p.hmax[n], xm[n & 1], xm[(n + 1) & 1], y.M1, p.B, p.ch0, p.wave,
+      e = launch_tcr_rows(p.scratch, p.hhalf[n], p.hmax[n], xm[n & 1], xm[(n + 1) & 1], y.M1, p.B, p.ch0, p.wave,
                           s);
     else
       e = launch_row<LOGMV, kPairConv, HT>(p.scratch, p.hh.p[n], p.tables, y.M1, p.B, p.ch0, p.wave, s);

@@ -60,6 +60,7 @@ struct FourStepLaunch {
   bool tcr;
   unsigned* xmax;
   const float* hmax[kMaxOrder];   // per filter: the spectrum block's per-channel maxima
+  const uint32_t* hhalf[kMaxOrder];   // per filter: the spectrum block's f16 copy (__half2 words)
 };
 
 // Records e as this thread's last CUDA error (hyena_last_cuda_error) and
@@ -110,9 +111,11 @@ cudaError_t launch_exp_sum_filter(const float* R, const float* lam, int d, int D
 cudaError_t launch_fourstep_wave(const FourStepLaunch& p, const Layout& y, cudaStream_t s);
 int fourstep_read_and_clear_timeout();
 // tensor-core row pass of one four-step stage (rows of 4096 points)
-cudaError_t launch_tcr_rows(float2* scr, const float2* spec, const float* hmax, const unsigned* xmax,
+cudaError_t launch_tcr_rows(float2* scr, const uint32_t* spec16, const float* hmax, const unsigned* xmax,
                             unsigned* xmax_clear, int M1, int B, long long ch0, int wave, cudaStream_t s);
 cudaError_t launch_tcr_hmax(const float2* spec, int D, int M, float* hmax, cudaStream_t s);
+// f16 copy of a spectrum block's bins for the row pass (after launch_tcr_hmax)
+cudaError_t launch_tcr_half(const float2* spec, const float* hmax, int D, int M, uint32_t* out, cudaStream_t s);
 int tcr_read_and_clear_timeout();
 cudaError_t launch_fourstep_spectrum(const float* h, float2* spec, const float2* tables, int D,
                                      const Layout& y, cudaStream_t s);

@@ -105,12 +105,16 @@ inline size_t tables_offset(const Layout& y, int D) {
 }
 // Four-step layouts with rows of 4096 points may run their row pass on the
 // tensor cores; their spectrum block ends with each channel's largest
-// spectrum component ([D] float, padded to float2), and their workspace holds
-// two words per channel beside the scratch (the column pass's per-channel maxima).
+// spectrum component ([D] float, padded to 16 bytes) and an f16 copy of the
+// spectrum ([D][M] __half2 in the same bin order, channel c times the power
+// of two f_c that puts its largest component in [2^14, 2^15)), whose rows the
+// row pass stages in shared memory. Their workspace holds two words per
+// channel beside the scratch (the column pass's per-channel maxima).
 inline bool tcr_layout(const Layout& y) { return y.fourstep && y.logMV == 12; }
 inline size_t hmax_offset(const Layout& y, int D) { return tables_offset(y, D) + y.table_len; }
+inline size_t tcr_half_offset(const Layout& y, int D) { return hmax_offset(y, D) + ((size_t)D + 3) / 4 * 2; }
 inline size_t spectrum_block_floats2(const Layout& y, int D) {
-  return hmax_offset(y, D) + (tcr_layout(y) ? (size_t)(D + 1) / 2 : 0);
+  return tcr_layout(y) ? tcr_half_offset(y, D) + (size_t)D * y.M / 2 : hmax_offset(y, D);
 }
 constexpr size_t kTcrChannelExtraBytes = 8;
 

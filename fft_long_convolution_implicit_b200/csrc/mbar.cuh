@@ -33,6 +33,25 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
+// L2 cache policy under which the lines a copy fills are the first to be
+// evicted: for data read once (filter spectrum rows), so that it does not
+// push out data that is read again (a wave's four-step scratch).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// bulk_g2s under an L2 cache policy
+__device__ __forceinline__ void bulk_g2s_policy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                                uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
+
 // Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, multiple of 16 bytes).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");

@@ -96,8 +96,12 @@ hyena_status hyena_filter_generate(const hyena_filter_params *p, int N, int D, i
 
 /*
  * Bytes of one filter's spectrum block for D channels and length L: the
- * spectrum in library order plus the FFT tables the forward reads. 0 when L
- * is unsupported or D < 1.
+ * spectrum in library order plus the FFT tables the forward reads, and the
+ * kernel-specific copies of the tensor-core paths (L = 1024, 2048, 8192: a
+ * copy in the kernel's bin order; L = 2^19 and 2^20: each channel's largest
+ * spectrum component, [D] float padded to 16 bytes, then an f16 copy of the
+ * spectrum, [D][L] __half2 at the end of the block). 0 when L is unsupported
+ * or D < 1.
  */
 size_t hyena_filter_spectrum_bytes(int D, int L);
 

@@ -138,3 +138,30 @@ def test_power_of_two_scaling_and_timeouts(hy):
     hy.check_device_timeouts()
     assert torch.equal(y1, y1b)
     assert torch.equal(y4, y1 * 4)
+
+
+@pytest.mark.parametrize("L,D", [(1 << 19, 3), (1 << 20, 2)])
+def test_row_pass_spectrum_copy(hy, L, D):
+    """Rows of 4096 (L = 2^19, 2^20): the spectrum block ends with each
+    channel's largest spectrum component ([D] float, padded to 16 bytes) and
+    an f16 copy of the bins ([D][L] __half2); the copy is f_c times the
+    float32 bins rounded to nearest, f_c the power of two that puts the
+    channel's largest component in [2^14, 2^15)."""
+    import torch
+    rng = np.random.default_rng(L + D)
+    h = (rng.standard_normal((D, L)) * np.exp(-np.arange(L) / (L / 8))).astype(np.float32)
+    hh = hy.filter_rfft(torch.from_numpy(h).cuda())
+    torch.cuda.synchronize()
+    blk = hh.cpu().numpy()
+    assert blk.size == hy.filter_spectrum_bytes(D, L)
+    half = blk[blk.size - 4 * D * L:].view(np.float16).reshape(D, 2 * L)
+    hmax_at = blk.size - 4 * D * L - 16 * ((D + 3) // 4)
+    hmax = blk[hmax_at: hmax_at + 4 * D].view(np.float32)
+    bins = blk[: 8 * D * L].view(np.float32).reshape(D, 2 * L)
+    for c in range(D):
+        top = np.abs(bins[c]).max()
+        assert hmax[c] == top, (c, hmax[c], top)
+        f_c = 2.0 ** (14 - np.floor(np.log2(top)))
+        assert 2.0 ** 14 <= top * f_c < 2.0 ** 15
+        want = (bins[c].astype(np.float64) * f_c).astype(np.float32).astype(np.float16)
+        assert np.array_equal(half[c].view(np.uint16), want.view(np.uint16)), c
