@@ -268,7 +268,10 @@ row_kernel(float2* __restrict__ scr, const float2* __restrict__ spec, const floa
       HA = HB = RS::bulk ? hs + MV : H + (size_t)(M1 / 2) * MV;
     }
     if constexpr (RS::bulk) {
-      if (!mbar_wait(smem_u32(&hbar), 0)) atomicExch(&g_fourstep_timeout, 1);
+      if (!mbar_wait(smem_u32(&hbar), 0)) {
+        atomicExch(&g_fourstep_timeout, 1);
+        mbar_wait(smem_u32(&hbar), 0, 1000000000ull);   // bounded second wait for the copies in flight
+      }
       paired_pass<LOGMV, MODE, true, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB, 1.0f / (8.0f * (float)M));
     } else {
       paired_pass<LOGMV, MODE, false, HT>(bA, bB, jA, jB, head, tw, Wv, rho, has_rho, HA, HB,

@@ -279,8 +279,9 @@ tcr_row_kernel(float2* __restrict__ scr, const uint32_t* __restrict__ spec16, co
     // the spectrum rows from shared memory (row B of a self-mirrored item is
     // row A)
     if (!mbar_wait(hbar, hphase)) {
-      ok = false;
+      ok = false;   // the next level barrier ends the kernel
       atomicExch(&g_tcr_timeout, 1);
+      mbar_wait(hbar, hphase, 1000000000ull);   // bounded second wait for the copies in flight
     }
     hphase ^= 1;
     h_pending = false;
