@@ -48,6 +48,14 @@ def test_host_queries(lib):
     assert hy.spectrum_layout(16)[0] == 128                  # small L is zero-extended to 128 points
     M, M1, MV = hy.spectrum_layout(1 << 20)
     assert M == 1 << 20 and M1 * MV == M and MV <= 4096
+    # rows of 4096 (L = 2^19, 2^20): spectrum, tables (MV-point plan, w_2MV, M1-point
+    # plan), [D] float maxima padded to 16 bytes, then the [D][L] __half2 copy
+    for L in (1 << 19, 1 << 20):
+        M, M1, MV = hy.spectrum_layout(L)
+        assert MV == 4096
+        for D in (1, 3, 4, 5):
+            tables = 8 * (2 * MV + M1)
+            assert hy.filter_spectrum_bytes(D, L) == 8 * D * M + tables + 16 * ((D + 3) // 4) + 4 * D * L
     M, M1, MV = hy.spectrum_layout(131072)
     assert (M1, MV) == (128, 1024)
     assert hy.forward_workspace_bytes(4, 768, 2048, 2, True) == 0
