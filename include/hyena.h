@@ -348,13 +348,16 @@ hyena_status hyena_filter_exponential(const float *R, const float *lambda, int d
 /*
  * Kernels that wait on mbarriers for asynchronous copies or tensor-core
  * completions (the striped bulk-copy kernel of hyena_striped_forward, taken
- * when a row's byte length is a multiple of 16, and the tcgen05 forward of
- * hyena_forward for bf16, B even, L = 8192, N <= 3) bound every wait in time: a
- * wait gives up 0.2 s of GPU global time after it started (each polling
- * step suspends for at most 20 us). A wait that runs out makes every thread
- * block of that launch stop early (its outputs are then invalid) and sets a
- * sticky flag on the current device; before exiting, such a block waits at
- * most 1 s more for the copies or tensor-core work it still has in flight.
+ * when a row's byte length is a multiple of 16; in hyena_forward the tcgen05
+ * kernel for bf16, B even, L = 8192, N <= 3, and the four-step row passes,
+ * whose spectrum rows arrive by bulk copies: rows of 1024 points, and the
+ * tcgen05 rows of 4096 points for bf16, N <= 3, L = 2^19 and 2^20) bound every
+ * wait in time: a wait gives up 0.2 s of GPU global time after it started
+ * (each polling step suspends for at most 20 us). A wait that runs out sets a
+ * sticky flag on the current device and the outputs of that launch are then
+ * invalid; the block waits at most 1 s more for the copies or tensor-core
+ * work it still has in flight, then stops early (the striped and tcgen05
+ * kernels) or finishes its item (the rows of 1024) and exits.
  * This call synchronises with the device, reads and clears the flag:
  * HYENA_OK if no wait ran out since the last call, HYENA_ERR_TIMEOUT
  * otherwise (HYENA_ERR_CUDA if it cannot be read).
