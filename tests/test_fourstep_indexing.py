@@ -1,6 +1,7 @@
-"""Bounds and coverage of the four-step kernels' global-memory indexing,
-replayed on the CPU over their launch grids (no GPU; the device sanitizer is
-not available, so this is the bounds evidence for the scratch indexing).
+"""Bounds and coverage of the global-memory indexing of the four-step kernels
+and of the tcgen05 pair kernel, replayed on the CPU over their launch grids
+(no GPU; the device sanitizer is not available, so this is the bounds
+evidence for their indexing).
 
 For each layout of the four-step path (L = 2^15 .. 2^20, from the library's
 own hyena_spectrum_layout), the index formulas of
@@ -9,8 +10,9 @@ own hyena_spectrum_layout), the index formulas of
 - tcr_row_kernel (csrc/tc_rows.cu): the scratch elements of a row pair each
   thread reads and writes, the spectrum bins of the product and their mirror
   partners, and the row pairs the items of a channel cover,
-are enumerated for every thread of the launch and checked to stay inside the
-buffers and to touch every element exactly once. The formulas are restated
+and of tcg_forward_kernel (csrc/tc_gemm.cu, L = 8192) are enumerated for
+every thread of the launch and checked to stay inside the buffers and to
+touch every element exactly once. The formulas are restated
 from the kernels; a change to a kernel's indexing must be made here too.
 """
 import numpy as np
@@ -116,3 +118,29 @@ def test_tensor_row_pass_indexing(L):
         for k in ((kA, kB) if kind == 0 else (kA,)):
             off_bytes = 4 * k * MV
             assert off_bytes % 16 == 0 and off_bytes + 4 * MV <= 4 * M
+
+
+def test_tcgen05_pair_kernel_indexing():
+    """tcg_forward_kernel (csrc/tc_gemm.cu, L = 8192, 256 threads, warp w, lane
+    l, q = w & 3, hw = w >> 2): the times t = l + 128 w + 32 i + 1024 n3
+    (i < 4, n3 < 8) of its v / gate loads and y stores, and the spectrum-copy
+    words (128 hw + 32 q + l + 256 t) * 32 + 16 hn + 4 k + e (t, hn < 2, k, e < 4)
+    of its product, each cover their row exactly once; 1 / f_c sits after the
+    2L words, inside the copy's row of 4 * 2L + 16 bytes."""
+    L = 8192
+    P = 2 * L
+    tid = np.arange(256)
+    w, l = tid >> 5, tid & 31
+    q, hw = w & 3, w >> 2
+    t = (l[:, None, None] + 128 * w[:, None, None] + 32 * np.arange(4)[None, :, None]
+         + 1024 * np.arange(8)[None, None, :]).ravel()
+    assert t.min() >= 0 and t.max() < L
+    assert np.bincount(t, minlength=L).tolist() == [1] * L
+    r = 128 * hw + 32 * q + l
+    words = ((r[:, None, None, None, None] + 256 * np.arange(2)[None, :, None, None, None]) * 32
+             + 16 * np.arange(2)[None, None, :, None, None] + 4 * np.arange(4)[None, None, None, :, None]
+             + np.arange(4)[None, None, None, None, :]).ravel()
+    assert words.min() >= 0 and words.max() < P
+    assert np.bincount(words, minlength=P).tolist() == [1] * P
+    row_bytes = 4 * P + 16
+    assert 4 * P + 4 <= row_bytes and row_bytes % 16 == 0
