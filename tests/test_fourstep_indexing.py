@@ -7,6 +7,8 @@ For each layout of the four-step path (L = 2^15 .. 2^20, from the library's
 own hyena_spectrum_layout), the index formulas of
 - col_kernel (csrc/fourstep.cu): input/gate/output elements of a channel row
   and the scratch elements (row n1, column n2) each pass reads and writes, and
+- row_kernel (csrc/fourstep.cu): the rows of each CTA's pair and the
+  elements of a row each thread reads and writes,
 - tcr_row_kernel (csrc/tc_rows.cu): the scratch elements of a row pair each
   thread reads and writes, the spectrum bins of the product and their mirror
   partners, and the row pairs the items of a channel cover,
@@ -62,6 +64,28 @@ def test_column_pass_indexing(L):
     idx = (rows * MV + n2[:, None]).ravel()
     assert idx.min() >= 0 and idx.max() < M1 * MV
     assert np.bincount(idx, minlength=M1 * MV).tolist() == [1] * (M1 * MV)
+
+
+@pytest.mark.parametrize("L", LS)
+def test_simt_row_pass_indexing(L):
+    """row_kernel (csrc/fourstep.cu): CTA p < M1 / 2 of a channel transforms
+    rows kA = p and kB = M1 - p (CTA 0: rows 0 and M1 / 2); its 2 TV threads
+    (TV = MV / 16) read and write elements tl + r MV / 16 (r < 16) of their row,
+    and the staged spectrum rows are 16-byte aligned bulk copies."""
+    M, M1, MV = hy.spectrum_layout(L)
+    rows = np.zeros(M1, int)
+    for p in range(M1 // 2):
+        kA, kB = p, (M1 // 2 if p == 0 else M1 - p)
+        rows[kA] += 1
+        rows[kB] += 1
+        for k in (kA, kB):
+            for elem in (8, 4):      # float32 and f16 spectrum rows
+                assert (elem * k * MV) % 16 == 0 and (elem * MV) % 16 == 0
+    assert rows.tolist() == [1] * M1
+    TV = MV // 16
+    idx = (np.arange(TV)[:, None] + np.arange(16)[None, :] * (MV // 16)).ravel()
+    assert idx.min() >= 0 and idx.max() < MV
+    assert np.bincount(idx, minlength=MV).tolist() == [1] * MV
 
 
 def tcr_items(M1: int):
