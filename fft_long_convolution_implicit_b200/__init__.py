@@ -159,6 +159,19 @@ def _dev(t, name):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _check_spectra(hhats, D: int, L: int, f16: bool = False):
+    """Each spectrum block must hold at least the bytes the library reads for
+    (D, L): hyena_filter_spectrum_bytes, or its f16 counterpart."""
+    lib = load()
+    need = lib.hyena_filter_spectrum_bytes_f16(D, L) if f16 else lib.hyena_filter_spectrum_bytes(D, L)
+    if need == 0:
+        return   # unsupported (D, L): the library call reports it
+    for n, hh in enumerate(hhats):
+        have = hh.numel() * hh.element_size()
+        if have < need:
+            raise ValueError(f"spectrum block {n} holds {have} bytes; (D={D}, L={L}) needs {need}")
+
+
 # ------------------------------------------------------------------ queries --
 
 def abi_version() -> int:
@@ -234,6 +247,7 @@ def forward(v, xs, hhats, y=None, workspace=None, stream=None):
     N = len(xs)
     if len(hhats) != N:
         raise ValueError("need one spectrum per gate")
+    _check_spectra(hhats, D, L)
     code = _dtype_code(v)
     for x in xs:
         if x.shape != v.shape or x.dtype != v.dtype:
@@ -274,6 +288,7 @@ def forward_f16_spectra(v, xs, hhats16, y=None, workspace=None, stream=None):
     N = len(xs)
     if len(hhats16) != N:
         raise ValueError("need one spectrum per gate")
+    _check_spectra(hhats16, D, L, f16=True)
     code = _dtype_code(v)
     for x in xs:
         if x.shape != v.shape or x.dtype != v.dtype:
@@ -303,6 +318,7 @@ def forward_static_workspace(v, xs, hhats, y=None, stream=None):
     N = len(xs)
     if len(hhats) != N:
         raise ValueError("need one spectrum per gate")
+    _check_spectra(hhats, D, L)
     code = _dtype_code(v)
     if y is None:
         y = torch.empty_like(v)
@@ -322,6 +338,7 @@ def backward(v, xs, hhats, dy, dv=None, dxs=None, dh=None, workspace=None, strea
     N = len(xs)
     if len(hhats) != N:
         raise ValueError("need one spectrum per gate")
+    _check_spectra(hhats, D, L)
     code = _dtype_code(v)
     for t in list(xs) + [dy]:
         if t.shape != v.shape or t.dtype != v.dtype:
@@ -463,6 +480,9 @@ class PreparedForward:
         torch = _torch()
         B, D, L = v.shape
         N = len(xs)
+        if len(hhats) != N:
+            raise ValueError("need one spectrum per gate")
+        _check_spectra(hhats, D, L, f16=f16_spectra)
         code = _dtype_code(v)
         self.y = torch.empty_like(v) if y is None else y
         need = forward_workspace_bytes(B, D, L, N, code == HYENA_BF16)
@@ -493,6 +513,9 @@ class PreparedBackward:
         torch = _torch()
         B, D, L = v.shape
         N = len(xs)
+        if len(hhats) != N:
+            raise ValueError("need one spectrum per gate")
+        _check_spectra(hhats, D, L)
         code = _dtype_code(v)
         self.dv = torch.empty_like(v) if dv is None else dv
         self.dxs = [torch.empty_like(v) for _ in range(N)] if dxs is None else list(dxs)

@@ -246,3 +246,19 @@ def test_header_is_plain_c_and_links_from_c(lib, tmp_path):
     assert int(out[2]) == lib.hyena_filter_spectrum_bytes_f16(768, 2048)
     assert int(out[3]) == lib.hyena_nd_spectrum_bytes(4, 2, I2(64, 64), 0)
     assert tuple(int(t) for t in out[4:7]) == hy.spectrum_layout(131072)
+
+
+def test_binding_rejects_short_spectrum_blocks():
+    """The binding checks every spectrum block against the bytes the library
+    reads for (D, L) before anything reaches the device (CPU tensors here)."""
+    import torch
+    v = torch.zeros(1, 2, 1 << 19, dtype=torch.bfloat16)
+    xs = [torch.zeros_like(v)]
+    short = [torch.zeros(hy.filter_spectrum_bytes(2, 1 << 19) - 16, dtype=torch.uint8)]
+    for call in (lambda: hy.forward(v, xs, short), lambda: hy.forward_static_workspace(v, xs, short),
+                 lambda: hy.backward(v, xs, short, v), lambda: hy.PreparedForward(v, xs, short)):
+        with pytest.raises(ValueError, match="spectrum block 0"):
+            call()
+    short16 = [torch.zeros(hy.load().hyena_filter_spectrum_bytes_f16(2, 1 << 19) - 16, dtype=torch.uint8)]
+    with pytest.raises(ValueError, match="spectrum block 0"):
+        hy.forward_f16_spectra(v, xs, short16)
